@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the LM-head loss path: one step = the five calls
+lmhead_fwd -> ce_fwd -> ce_bwd (BF16 dlogits) -> lmhead_bwd_dx -> lmhead_bwd_dw
+on one synthetic batch (M=1024 tokens, K=4096, V=32768; X ~ N(0,1),
+W ~ N(0,0.02^2) in BF16, 2% of targets ignored, grad_loss = 1/num_valid).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  Timing: CUDA events on the launching stream
+around every step (and every call inside it), L2 flushed by a 512 MiB write
+between steps outside the timed events, device time summed over the K steps
+and the maximum taken over ranks.  With N > 1 (torchrun) every rank runs an
+independent replica of the step on its own batch (weak scaling, no
+collective on the data path).
+
+--impl reference times the CPU oracle (FP64, all host cores) on a bounded
+sample of the same workload; it is the deliberately slow baseline, not a
+competitor.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LM-head+CE fwd+bwd tokens/s; GEMM TFLOP/s and CE GB/s as % of B200 peak"
+WORKLOAD = dict(name="lmhead_1024x4096x32768", M=1024, K=4096, V=32768)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("lm_head_fp32_b200/csrc/gemm_tc.cuh", "lm_head_fp32_b200/csrc/ce_kernels.cuh",
+                  "lm_head_fp32_b200/csrc/ptx.cuh", "lm_head_fp32_b200/csrc/lmhead.cu")
+FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample", type=int, default=96,
+                    help="tokens of the workload the CPU oracle baseline processes")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """Per-launch DRAM bytes of each kernel from the committed ncu summary, or
+    {} when that summary was taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic_lmhead_1024x4096x32768.md")
+    if not os.path.exists(p):
+        return {}
+    txt = open(p).read()
+    m = re.search(r"kernel-source-hash:\s*([0-9a-f]+)", txt)
+    if not m or m.group(1) != kernel_source_hash():
+        return {}
+    out = {}
+    for name, val in re.findall(r"^\|\s*(\w+)\s*\|\s*([0-9.eE+]+)\s*\|", txt, flags=re.M):
+        try:
+            out[name] = float(val)
+        except ValueError:
+            pass
+    return out
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    """Maximum of a per-rank float across all ranks (the job's device time)."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle baseline (the reference arm of this path)
+# ----------------------------------------------------------------------------
+
+def oracle_step(X, W, t, g, rows):
+    """The whole path on the CPU oracle for the given token rows: logits,
+    CE forward, CE backward (BF16 round), dX rows and those tokens' share of dW."""
+    import numpy as np
+    import oracle
+    from lm_head_fp32_b200 import synth
+    xb, wb = synth.bf16_bits(X), synth.bf16_bits(W)
+    L = oracle.round_f32(oracle.logits(xb, wb, rows=rows))
+    tt = t.numpy()[rows]
+    oracle.ce_fwd(L, tt)
+    dl = oracle.round_bf16(oracle.ce_bwd(L, tt, g))
+    oracle.dx(dl, wb)                       # dX for the sampled rows
+    oracle.dw(dl, xb[rows])                 # their contribution to dW (all V rows)
+
+
+def cpu_baseline(cfg, X, W, t, g, tokens: int):
+    import numpy as np
+    import oracle
+    rows = np.arange(tokens, dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle_step(X, W, t, g, rows)
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{tokens} of {cfg.M} tokens of {cfg.name} through all five steps "
+                      f"(logits, CE fwd, CE bwd, dX rows, their dW share), FP64, {dt:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, local, pg = dist_setup(args)
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    from lm_head_fp32_b200 import synth
+    cfg = synth.MIDSIZE
+    X, W, t = cfg.make()
+    g = cfg.grad_scalar(t)
+    import numpy as np
+    import oracle
+    per_step = max(1, min(args.cpu_sample, 16))
+    for i in range(args.warmup):
+        oracle_step(X, W, t, g, np.arange(per_step, dtype=np.int64) + (i * per_step) % cfg.M)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(X, W, t, g, (np.arange(per_step, dtype=np.int64) + i * per_step) % cfg.M)
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "V": cfg.V,
+                       "tokens_per_step": per_step},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"{per_step} tokens of {cfg.name} per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    from lm_head_fp32_b200 import lmhead, synth
+
+    world, rank, local, pg = dist_setup(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = synth.MIDSIZE
+    M, K, V = cfg.M, cfg.K, cfg.V
+    # every rank draws its own batch (replica r uses seed + 7919 r)
+    rcfg = synth.GemmConfig(cfg.name, M, K, V, cfg.dist, cfg.x_std, cfg.w_std, cfg.ignore_frac,
+                            cfg.grad, cfg.seed + 7919 * rank)
+    X, W, t = rcfg.make()
+    g = rcfg.grad_scalar(t)
+    Xd, Wd, td = X.to(dev), W.to(dev), t.to(dev)
+    gd = torch.tensor([g], dtype=torch.float32, device=dev)
+    logits = torch.empty((M, V), dtype=torch.float32, device=dev)
+    stats = torch.empty((M, 4), dtype=torch.float32, device=dev)
+    dl = torch.empty((M, V), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.float32, device=dev)
+    dW = torch.empty((V, K), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    names = ["lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw"]
+    calls = [
+        lambda: lmhead.lmhead_fwd(Xd, Wd, logits, status),
+        lambda: lmhead.ce_fwd(logits, td, stats, -100, status),
+        lambda: lmhead.ce_bwd(logits, td, stats, gd, dl, -100, status),
+        lambda: lmhead.lmhead_bwd_dx(dl, Wd, dX, status),
+        lambda: lmhead.lmhead_bwd_dw(dl, Xd, dW, status),
+    ]
+
+    def step():
+        for c in calls:
+            c()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K_steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(pg)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)                      # let the sampler attach
+    for i in range(K_steps):
+        flush.zero_()                     # L2 flush, outside the timed events
+        e = ev[i]
+        e[0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            e[j + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(pg)
+    per_call = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_steps)] for j in range(len(calls))]
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(K_steps)]
+    total_ms = max_over_ranks(sum(step_ms), pg, dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    value = world * M * K_steps / (total_ms / 1e3)
+
+    # end to end through the public API: pinned host X and targets in, loss out
+    Xh = X.pin_memory()
+    th = t.pin_memory()
+    lossh = torch.empty((M, 4), dtype=torch.float32).pin_memory()
+    e2e_steps = max(10, min(K_steps, 50))
+    for _ in range(3):
+        Xd.copy_(Xh, non_blocking=True)
+        td.copy_(th, non_blocking=True)
+        step()
+        lossh.copy_(stats, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for _ in range(e2e_steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Xd.copy_(Xh, non_blocking=True)
+        td.copy_(th, non_blocking=True)
+        step()
+        lossh.copy_(stats, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    e2e_ms = max_over_ranks(e2e_ms, pg, dev)
+    h2d = Xh.numel() * Xh.element_size() + th.numel() * th.element_size()
+    d2h = lossh.numel() * lossh.element_size()
+
+    # roofline of every kernel; the dominant one goes in "roofline"
+    peaks, peak_src = load_peaks()
+    flop = 2.0 * M * K * V
+    nv = int((t != -100).sum())
+    ce_fwd_bytes = nv * V * 4 + M * (8 + 16)
+    ce_bwd_bytes = nv * V * 4 + M * V * 2 + M * (8 + 16)
+    algo = {"lmhead_fwd": ("tensor", flop), "ce_fwd": ("hbm", ce_fwd_bytes),
+            "ce_bwd": ("hbm", ce_bwd_bytes), "lmhead_bwd_dx": ("tensor", flop),
+            "lmhead_bwd_dw": ("tensor", flop)}
+    traffic = committed_traffic()
+    kernels = {}
+    for j, n in enumerate(names):
+        ms = statistics.mean(per_call[j])
+        bound, work = algo[n]
+        if bound == "tensor":
+            ach, peak, unit = work / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        else:
+            ach, peak, unit = work / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        kernels[n] = {"ms": round(ms, 5), "bound": bound, "achieved": round(ach, 1), "unit": unit,
+                      "frac": round(ach / peak, 4), "algorithmic": work}
+    dom = max(names, key=lambda n: kernels[n]["ms"])
+    kd = kernels[dom]
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"],
+                "peak": peaks["bf16_tflops"] if kd["bound"] == "tensor" else peaks["hbm_gbs"],
+                "unit": kd["unit"], "frac": kd["frac"], "peak_source": f"{peak_src} (burst)",
+                "traffic": traffic.get(dom)}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K_steps, "warmup": args.warmup, "ms_per_step": total_ms / K_steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "M": M, "K": K, "V": V, "logits": "fp32",
+                       "dlogits": "bf16", "dX_dW": "fp32", "accumulate": "fp32",
+                       "ignored_rows": M - nv, "grad_loss": "1/num_valid",
+                       "l2": "flushed between steps (512 MiB write outside the timed events)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline, "kernels": kernels,
+            "e2e": {"value": world * M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(calls) * K_steps, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, X, W, t, g, args.cpu_sample)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

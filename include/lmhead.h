@@ -1,0 +1,151 @@
+/*
+ * lmhead.h -- C ABI of the B200 (sm_100a) LM-head loss path.
+ *
+ * The library computes, on one GPU:
+ *   lmhead_fwd     logits[M,V] = X[M,K] . W[V,K]^T, FP32 accumulator stored
+ *                  unrounded (or a BF16 copy of it, for comparison)
+ *   ce_fwd         per-row cross-entropy statistics {m, d, x_y, loss}
+ *   ce_bwd         dlogits = (softmax - onehot(target)) * grad_loss, in FP32,
+ *                  rounded to the output dtype only at the store
+ *   lmhead_bwd_dx  dX[M,K] = dlogits[M,V] . W[V,K]
+ *   lmhead_bwd_dw  dW[V,K] = dlogits[M,V]^T . X[M,K]
+ *
+ * Sources (page title, section):
+ *   [P1] Megatron-LM PR #6252 "Add mixed-precision (FP32) LM output logits":
+ *        "What does this PR do?" (FP32 GEMM output instead of BF16-rounded
+ *        logits; gradients cast back to BF16 under the GEMM contract),
+ *        "Tests" (only bf16 and fp32 logit dtypes are accepted, fp16 is
+ *        rejected), "Integer bitwise exactness results".
+ *   [P2] TransformerEngine #2325 "[Pytorch] change fused cross entropy
+ *        backward grad to fp32 and reduce one read": "Description" and
+ *        "Changes" (backward computed in FP32, one fewer read of the logits)
+ *        and the review discussion (the forward saves the target, n_rows x 1,
+ *        and m_d_X_y, n_rows x 4).
+ *
+ * Conventions shared by every call
+ *   - All array arguments are DEVICE pointers into row-major, contiguous
+ *     buffers owned by the caller.  The library allocates nothing, keeps no
+ *     per-call state and never synchronises: every call only enqueues work on
+ *     `stream` (NULL = legacy default stream) and returns.
+ *   - BF16 data is IEEE binary32's upper 16 bits; FP32 is IEEE binary32.
+ *   - Errors are returned, never raised: arguments are validated on the host
+ *     before anything is launched, and a failing launch maps to LMH_ERR_CUDA.
+ *   - `status` (nullable) is a device int32 word that kernels OR condition
+ *     bits into (LMH_DEV_*).  The caller zeroes it, and reads it after the
+ *     stream has been synchronised.  Nothing is trapped on the device.
+ *   - Sizes are int64; every size must be >= 1 unless stated otherwise.
+ */
+#ifndef LMHEAD_H_
+#define LMHEAD_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported from liblmhead.so (everything else in the library is hidden). */
+#if defined(__GNUC__)
+#define LMH_API __attribute__((visibility("default")))
+#else
+#define LMH_API
+#endif
+
+/* Host-side result of a call. */
+typedef enum {
+    LMH_OK = 0,
+    LMH_ERR_INVALID_ARG = 1,  /* null pointer, size < 1, size too large   */
+    LMH_ERR_MISALIGNED = 2,   /* pointer or row stride breaks the layout  */
+    LMH_ERR_UNSUPPORTED = 3,  /* dtype or stride value not supported      */
+    LMH_ERR_CUDA = 4          /* the CUDA runtime reported an error       */
+} lmh_status_t;
+
+/* Element types.  As with the logit-dtype option of [P1] "Tests", only FP32
+ * and BF16 are accepted; LMH_F16 (and any other value) is rejected with
+ * LMH_ERR_UNSUPPORTED. */
+typedef enum { LMH_F32 = 0, LMH_BF16 = 1, LMH_F16 = 2 } lmh_dtype_t;
+
+/* Bits ORed into *status by the kernels. */
+#define LMH_DEV_BAD_TARGET 0x1   /* a target neither ignore_index nor in [0,V);
+                                    the row was treated as ignored          */
+#define LMH_DEV_PIPE_TIMEOUT 0x2 /* a pipeline wait gave up (bounded spin);
+                                    the output of that call is not valid    */
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *lmh_stream_t;
+
+/* logits = X . W^T  ([P1] "What does this PR do?").
+ *   X       [M,K] BF16, K contiguous.         W [V,K] BF16, K contiguous.
+ *   logits  [M,V] FP32 (out_dtype LMH_F32: the accumulator, unrounded) or
+ *           BF16 (LMH_BF16: the accumulator rounded to nearest even).
+ *   Requirements: K % 8 == 0 (16-byte rows for the tensor-memory copies),
+ *   X and W 16-byte aligned, logits 4-byte aligned; M, V, K <= 2^31 - 1.
+ *   Accumulation is FP32 inside the tensor cores; when every partial sum is
+ *   an exactly representable integer (BF16 integers in [-8,8] with
+ *   K * 64 < 2^24, [P1] "Integer bitwise exactness results") the FP32 output
+ *   is exact.  Deterministic: repeated calls give identical bits. */
+LMH_API lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_dtype,
+                        int64_t M, int64_t K, int64_t V, int32_t *status,
+                        lmh_stream_t stream);
+
+/* Cross-entropy forward statistics ([P2] discussion: target and m_d_X_y).
+ *   logits  [M,V] FP32.   target [M] int64.
+ *   stats   [M,4] FP32, per row {m, d, x_y, loss}:
+ *             m = max_j x_j, d = sum_j exp(x_j - m), x_y = x[target],
+ *             loss = m + log(d) - x_y  (= -log softmax(x)_target).
+ *   A row whose target equals ignore_index is not read and gets
+ *   {0,0,0,0}.  A target outside [0,V) that is not ignore_index sets
+ *   LMH_DEV_BAD_TARGET in *status and the row is treated as ignored.
+ *   Any V >= 1; no alignment beyond the element size. */
+LMH_API lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats,
+                    int64_t M, int64_t V, int64_t ignore_index, int32_t *status,
+                    lmh_stream_t stream);
+
+/* Cross-entropy backward in FP32 ([P2] "Description", "Changes"; the BF16
+ * cast at the end is the one of [P1] "What does this PR do?").
+ *   logits     [M,V] FP32, the same buffer ce_fwd read.
+ *   target     [M] int64.   stats [M,4] FP32 from ce_fwd.
+ *   grad_loss  FP32 upstream gradient of the per-row loss:
+ *              grad_loss_stride 0 = one scalar for every row,
+ *              1 = one value per row ([M]); anything else is unsupported.
+ *   dlogits    [M,V], dl_dtype LMH_F32 or LMH_BF16 (round to nearest even):
+ *              dl[i,j] = (exp(x_ij - m_i) / d_i - [j == target_i]) * g_i.
+ *              Ignored and bad-target rows are written as zeros.
+ *              With LMH_F32, dlogits may be the logits buffer itself
+ *              (in-place; each element is read before it is overwritten).
+ *   Any V >= 1. */
+LMH_API lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *stats,
+                    const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
+                    int32_t dl_dtype, int64_t M, int64_t V, int64_t ignore_index,
+                    int32_t *status, lmh_stream_t stream);
+
+/* dX = dlogits . W, the input gradient of logits = X . W^T
+ * ([P1] "What does this PR do?", backward under the GEMM contract).
+ *   dlogits [M,V] BF16.  W [V,K] BF16.
+ *   dX      [M,K] FP32 (LMH_F32) or BF16 (LMH_BF16).
+ *   Requirements: V % 8 == 0 and K % 8 == 0 (16-byte rows), inputs 16-byte
+ *   aligned.  Deterministic. */
+LMH_API lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t out_dtype,
+                           int64_t M, int64_t K, int64_t V, int32_t *status,
+                           lmh_stream_t stream);
+
+/* dW = dlogits^T . X, the weight gradient of logits = X . W^T.
+ *   dlogits [M,V] BF16.  X [M,K] BF16.
+ *   dW      [V,K] FP32 (LMH_F32) or BF16 (LMH_BF16).
+ *   Requirements: V % 8 == 0 and K % 8 == 0, inputs 16-byte aligned.
+ *   Deterministic. */
+LMH_API lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t out_dtype,
+                           int64_t M, int64_t K, int64_t V, int32_t *status,
+                           lmh_stream_t stream);
+
+/* Static, NUL-terminated description of a status value. */
+LMH_API const char *lmh_status_string(lmh_status_t s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+LMH_API int32_t lmh_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMHEAD_H_ */

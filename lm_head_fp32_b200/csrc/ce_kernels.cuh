@@ -1,0 +1,280 @@
+// ce_kernels.cuh -- cross-entropy forward statistics and FP32 backward.
+//
+// TransformerEngine #2325 "[Pytorch] change fused cross entropy backward grad
+// to fp32 and reduce one read": the forward makes one pass over each row of
+// FP32 logits and saves only the target and m_d_X_y (n_rows x 4) instead of
+// writing gradients; the backward recomputes softmax from the saved (m, d) in
+// FP32 and writes the gradient, so each kernel reads the logits once.
+//
+// Both kernels are HBM-bound row sweeps: one CTA per row (grid-stride over
+// rows), 128-bit read-only streaming loads, an online (max, sum-exp) pair per
+// thread merged by warp shuffles and then across warps in shared memory.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace lmh {
+
+constexpr int kCeThreads = 512;
+constexpr float kLog2e = 1.4426950408889634f;  // 1 / ln 2
+
+struct MaxSum {
+    float m;  // running maximum
+    float d;  // sum of exp(x - m)
+};
+
+// exp(t) for t <= 0, via the hardware base-2 exponential.
+__device__ __forceinline__ float exp_neg(float t) { return exp2f(t * kLog2e); }
+
+// Merge two (max, sum-exp) pairs: the associative step of the online softmax.
+__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b)
+{
+    if (a.m < b.m) {
+        MaxSum t = a;
+        a = b;
+        b = t;
+    }
+    // a.m >= b.m; b.m == -inf means b holds nothing
+    if (b.m == -INFINITY)
+        return a;
+    return MaxSum{a.m, a.d + b.d * exp_neg(b.m - a.m)};
+}
+
+// Fold a batch of N values into the running pair: one rescale per batch,
+// and the batch's own exponentials are summed first (short partial sums).
+template <int N>
+__device__ __forceinline__ void fold(MaxSum &s, const float (&v)[N])
+{
+    float mx = v[0];
+#pragma unroll
+    for (int i = 1; i < N; ++i)
+        mx = fmaxf(mx, v[i]);
+    if (mx > s.m) {
+        s.d = (s.m == -INFINITY) ? 0.f : s.d * exp_neg(s.m - mx);
+        s.m = mx;
+    }
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+        part += exp_neg(v[i] - s.m);
+    s.d += part;
+}
+
+__device__ __forceinline__ void fold1(MaxSum &s, float x)
+{
+    if (x > s.m) {
+        s.d = (s.m == -INFINITY) ? 0.f : s.d * exp_neg(s.m - x);
+        s.m = x;
+    }
+    s.d += exp_neg(x - s.m);
+}
+
+__device__ __forceinline__ float4 ldg_stream(const float4 *p)
+{
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float ldg_stream1(const float *p)
+{
+    float v;
+    asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// Coherent streaming loads, for a buffer the same kernel also writes (in-place).
+__device__ __forceinline__ float4 ld_cs(const float4 *p) { return __ldcs(p); }
+__device__ __forceinline__ float ld_cs1(const float *p) { return __ldcs(p); }
+
+template <bool ALIAS>
+__device__ __forceinline__ float4 load4(const float4 *p) { return ALIAS ? ld_cs(p) : ldg_stream(p); }
+template <bool ALIAS>
+__device__ __forceinline__ float load1(const float *p) { return ALIAS ? ld_cs1(p) : ldg_stream1(p); }
+
+// Block-wide merge of every thread's pair; the result is valid in all threads.
+__device__ __forceinline__ MaxSum block_merge(MaxSum s, MaxSum *red /* [32] */)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        MaxSum t{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.d, o)};
+        s = merge(s, t);
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0)
+        red[warp] = s;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        s = lane < nw ? red[lane] : MaxSum{-INFINITY, 0.f};
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            MaxSum t{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.d, o)};
+            s = merge(s, t);
+        }
+        if (lane == 0)
+            red[0] = s;
+    }
+    __syncthreads();
+    s = red[0];
+    __syncthreads();  // red[] may be reused by the next row
+    return s;
+}
+
+// Row classification shared by both kernels: 0 valid, 1 ignored, 2 bad target.
+__device__ __forceinline__ int row_kind(int64_t y, int64_t V, int64_t ignore_index)
+{
+    if (y == ignore_index)
+        return 1;
+    if (y < 0 || y >= V)
+        return 2;
+    return 0;
+}
+
+// stats[row] = {m, d, x_y, loss}.  VEC: V % 4 == 0 and logits 16-byte aligned.
+template <bool VEC>
+__global__ void __launch_bounds__(kCeThreads) ce_fwd_kernel(const float *__restrict__ logits,
+                                                            const int64_t *__restrict__ target,
+                                                            float4 *__restrict__ stats, int64_t M,
+                                                            int64_t V, int64_t ignore_index,
+                                                            int32_t *status)
+{
+    __shared__ MaxSum red[32];
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const int64_t y = target[row];
+        const int kind = row_kind(y, V, ignore_index);
+        if (kind != 0) {
+            if (threadIdx.x == 0) {
+                stats[row] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (kind == 2 && status)
+                    atomicOr(status, 1);
+            }
+            continue;  // uniform across the block: no barrier skipped unevenly
+        }
+        const float *x = logits + row * V;
+        MaxSum s{-INFINITY, 0.f};
+        if (VEC) {
+            const float4 *x4 = reinterpret_cast<const float4 *>(x);
+            const int64_t n4 = V >> 2;
+            int64_t i = threadIdx.x;
+            // four 128-bit loads in flight per thread per step
+            for (; i + 3 * kCeThreads < n4; i += 4 * kCeThreads) {
+                float4 a = ldg_stream(x4 + i), b = ldg_stream(x4 + i + kCeThreads),
+                       c = ldg_stream(x4 + i + 2 * kCeThreads),
+                       e = ldg_stream(x4 + i + 3 * kCeThreads);
+                const float v[16] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w,
+                                     c.x, c.y, c.z, c.w, e.x, e.y, e.z, e.w};
+                fold<16>(s, v);
+            }
+            for (; i < n4; i += kCeThreads) {
+                float4 a = ldg_stream(x4 + i);
+                const float v[4] = {a.x, a.y, a.z, a.w};
+                fold<4>(s, v);
+            }
+        } else {
+            for (int64_t j = threadIdx.x; j < V; j += kCeThreads)
+                fold1(s, ldg_stream1(x + j));
+        }
+        s = block_merge(s, red);
+        if (threadIdx.x == 0) {
+            const float xy = x[y];
+            // (m - x_y) first: exact when x_y is the maximum, so a near-zero
+            // loss is not swamped by the rounding of m + log(d).
+            const float loss = (s.m - xy) + logf(s.d);
+            stats[row] = make_float4(s.m, s.d, xy, loss);
+        }
+    }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store4(OutT *p, float a, float b, float c, float d);
+
+template <>
+__device__ __forceinline__ void store4<float>(float *p, float a, float b, float c, float d)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+}
+
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, float a, float b, float c,
+                                                      float d)
+{
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&lo);
+    u.y = *reinterpret_cast<uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+
+__device__ __forceinline__ void store1(float *p, float a) { *p = a; }
+__device__ __forceinline__ void store1(__nv_bfloat16 *p, float a) { *p = __float2bfloat16_rn(a); }
+
+// dl[row, j] = (exp(x - m) / d - [j == y]) * g, FP32 arithmetic, rounded to
+// OutT only at the store.  Ignored / bad-target rows are written as zeros.
+// VEC: V % 4 == 0, logits 16-byte and dl (4 * sizeof(OutT))-byte aligned.
+// Each element is read before it is written, by the same thread, so dl may
+// alias logits when OutT is float (ALIAS: coherent loads instead of the
+// read-only path).
+template <typename OutT, bool VEC, bool ALIAS>
+__global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(
+    const float *logits, const int64_t *__restrict__ target, const float4 *__restrict__ stats,
+    const float *__restrict__ grad_loss, int64_t grad_stride, OutT *dl, int64_t M, int64_t V,
+    int64_t ignore_index, int32_t *status)
+{
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const int64_t y = target[row];
+        const int kind = row_kind(y, V, ignore_index);
+        const float *x = logits + row * V;
+        OutT *o = dl + row * V;
+        if (kind != 0) {
+            if (kind == 2 && status && threadIdx.x == 0)
+                atomicOr(status, 1);
+            if (VEC) {
+                for (int64_t i = threadIdx.x; i < (V >> 2); i += kCeThreads)
+                    store4<OutT>(o + 4 * i, 0.f, 0.f, 0.f, 0.f);
+            } else {
+                for (int64_t j = threadIdx.x; j < V; j += kCeThreads)
+                    store1(o + j, 0.f);
+            }
+            continue;
+        }
+        const float4 st = stats[row];
+        const float m = st.x;
+        const float inv_d = 1.0f / st.y;
+        const float g = grad_loss[row * grad_stride];
+        if (VEC) {
+            const float4 *x4 = reinterpret_cast<const float4 *>(x);
+            const int64_t n4 = V >> 2;
+            int64_t i = threadIdx.x;
+            for (; i + kCeThreads < n4; i += 2 * kCeThreads) {
+                const float4 a = load4<ALIAS>(x4 + i), b = load4<ALIAS>(x4 + i + kCeThreads);
+                const int64_t ja = 4 * i, jb = 4 * (i + kCeThreads);
+                store4<OutT>(o + ja, (exp_neg(a.x - m) * inv_d - (ja + 0 == y)) * g,
+                             (exp_neg(a.y - m) * inv_d - (ja + 1 == y)) * g,
+                             (exp_neg(a.z - m) * inv_d - (ja + 2 == y)) * g,
+                             (exp_neg(a.w - m) * inv_d - (ja + 3 == y)) * g);
+                store4<OutT>(o + jb, (exp_neg(b.x - m) * inv_d - (jb + 0 == y)) * g,
+                             (exp_neg(b.y - m) * inv_d - (jb + 1 == y)) * g,
+                             (exp_neg(b.z - m) * inv_d - (jb + 2 == y)) * g,
+                             (exp_neg(b.w - m) * inv_d - (jb + 3 == y)) * g);
+            }
+            for (; i < n4; i += kCeThreads) {
+                const float4 a = load4<ALIAS>(x4 + i);
+                const int64_t ja = 4 * i;
+                store4<OutT>(o + ja, (exp_neg(a.x - m) * inv_d - (ja + 0 == y)) * g,
+                             (exp_neg(a.y - m) * inv_d - (ja + 1 == y)) * g,
+                             (exp_neg(a.z - m) * inv_d - (ja + 2 == y)) * g,
+                             (exp_neg(a.w - m) * inv_d - (ja + 3 == y)) * g);
+            }
+        } else {
+            for (int64_t j = threadIdx.x; j < V; j += kCeThreads) {
+                const float v = load1<ALIAS>(x + j);
+                store1(o + j, (exp_neg(v - m) * inv_d - (j == y)) * g);
+            }
+        }
+    }
+}
+
+}  // namespace lmh

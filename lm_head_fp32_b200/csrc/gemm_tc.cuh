@@ -1,0 +1,306 @@
+// gemm_tc.cuh -- persistent tcgen05 GEMM for sm_100a with a direct FP32 (or
+// BF16) epilogue, used for the three contractions of the LM head:
+//
+//   logits[i, v] = sum_k X[i,k] W[v,k]        (A = W,   B = X,    both K-major)
+//   dX[i, k]     = sum_v dl[i,v] W[v,k]       (A = W^T  MN-major, B = dl K-major)
+//   dW[v, k]     = sum_i dl[i,v] X[i,k]       (A = X^T  MN-major, B = dl^T MN-major)
+//
+// Megatron-LM PR #6252 "Add mixed-precision (FP32) LM output logits", "What
+// does this PR do?": the vocabulary GEMM keeps its FP32 accumulator as the
+// output instead of rounding every logit to BF16.  Here the accumulator lives
+// in tensor memory and the epilogue stores it unrounded.
+//
+// Generic form: D[m, n] = sum_k A[m, k] B[n, k], stored at out[n * ldo + m].
+// The MMA's M dimension (128 lanes of tensor memory) is always the output's
+// contiguous dimension, so each epilogue warp stores 32 consecutive elements
+// (one 128-byte line for FP32) per instruction straight from registers.
+//
+// CTA roles (192 threads, one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: fills a STAGES-deep ring of A/B k-blocks
+//   warp 1      tensor-memory owner and MMA issuer (one elected thread)
+//   warps 2..5  epilogue: tensor memory -> registers -> global memory
+// Two accumulators of BN columns let the epilogue of tile t overlap the MMAs
+// of tile t+1.  Every wait is bounded (see mbar_wait); on a timeout the CTA
+// drains its own copies and MMAs, frees tensor memory, sets a status bit and
+// returns.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace lmh {
+
+constexpr int kGemmThreads = 192;
+constexpr int kBlockM = 128;  // MMA M: tensor-memory lanes
+constexpr int kBlockK = 64;   // one 128-byte swizzle row of BF16
+constexpr int kUmmaK = 16;    // K of one kind::f16 MMA
+
+struct GemmParams {
+    void *out;
+    int64_t ldo;        // elements between consecutive n of the output
+    int32_t Mdim;       // extent of m (output contiguous dim)
+    int32_t Ndim;       // extent of n
+    int32_t Kdim;       // reduction length
+    int32_t num_m_tiles;
+    int32_t num_n_tiles;
+    int32_t m_fastest;  // tile order: 1 = consecutive tiles share n (B panel)
+    int32_t *status;
+};
+
+template <int BN, bool A_MN, bool B_MN>
+struct GemmCfg {
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(!B_MN || BN % 64 == 0, "MN-major B is loaded in 64-wide boxes");
+    static constexpr int A_BYTES = kBlockM * kBlockK * 2;  // 16 KB
+    static constexpr int B_BYTES = BN * kBlockK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+    static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;
+    // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
+    static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+    static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + BAR_BYTES + 16;
+    static constexpr uint32_t IDESC = idesc_bf16_f32(kBlockM, BN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
+    static_assert(STAGES >= 2, "pipeline depth");
+};
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[32]);
+
+template <>
+__device__ __forceinline__ void tmem_ld_chunk<32>(uint32_t taddr, uint32_t (&r)[32])
+{
+    tmem_ld32(taddr, r);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_chunk<16>(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void store_out(float *p, uint32_t bits) { *p = __uint_as_float(bits); }
+__device__ __forceinline__ void store_out(__nv_bfloat16 *p, uint32_t bits)
+{
+    *p = __float2bfloat16_rn(__uint_as_float(bits));
+}
+
+__device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt, int &nt)
+{
+    if (p.m_fastest) {
+        mt = t % p.num_m_tiles;
+        nt = t / p.num_m_tiles;
+    } else {
+        nt = t % p.num_n_tiles;
+        mt = t / p.num_n_tiles;
+    }
+}
+
+template <int BN, bool A_MN, bool B_MN, typename OutT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p)
+{
+    using C = GemmCfg<BN, A_MN, B_MN>;
+    constexpr int S = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *tiles = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
+    uint64_t *full = bars;
+    uint64_t *empty = bars + S;
+    uint64_t *acc_full = bars + 2 * S;
+    uint64_t *acc_empty = bars + 2 * S + 2;
+    uint64_t *drain = bars + 2 * S + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+    const int num_kb = (p.Kdim + kBlockK - 1) / kBlockK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4 * 32);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1)
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_last();
+            const uint64_t pol_b = policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            int64_t issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                int mt, nt;
+                tile_coords(t, p, mt, nt);
+                const int m0 = mt * kBlockM, n0 = nt * BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = tiles + stage * C::STAGE_BYTES;
+                    uint8_t *sb = sa + C::A_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+                    const int k0 = kb * kBlockK;
+                    if (A_MN) {
+#pragma unroll
+                        for (int j = 0; j < kBlockM / 64; ++j)
+                            tma_load_2d(&tmA, &full[stage], sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
+                    } else {
+                        tma_load_2d(&tmA, &full[stage], sa, k0, m0, pol_a);
+                    }
+                    if (B_MN) {
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(&tmB, &full[stage], sb + j * 64 * kBlockK * 2, n0 + 64 * j, k0, pol_b);
+                    } else {
+                        tma_load_2d(&tmB, &full[stage], sb, k0, n0, pol_b);
+                    }
+                    ++issued;
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA exits
+                volatile int no_abort = 0;
+                for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i)
+                    mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1), &no_abort);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t acc = 0, acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(tiles + stage * C::STAGE_BYTES);
+                    const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+                        // K-major: advance 32 bytes along the swizzled row.
+                        // MN-major: advance 16 rows of 128 bytes.
+                        const uint64_t da = A_MN ? smem_desc_sw128(sa + k * 2048, 64 * kBlockK * 2, 1024)
+                                                 : smem_desc_sw128(sa + k * 32, 16, 1024);
+                        const uint64_t db = B_MN ? smem_desc_sw128(sb + k * 2048, 64 * kBlockK * 2, 1024)
+                                                 : smem_desc_sw128(sb + k * 32, 16, 1024);
+                        mma_bf16(d_tmem, da, db, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&empty[stage]);  // frees the smem slot when these MMAs finish
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // wait until every MMA issued by this thread has completed
+            mma_commit(drain);
+            volatile int no_abort = 0;
+            mbar_wait(drain, 0, &no_abort);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+        const int row = q * 32 + lane;
+        OutT *out = static_cast<OutT *>(p.out);
+        uint32_t acc = 0, acc_phase = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            // every lane waits, then the warp agrees, so the .sync.aligned
+            // tensor-memory loads below always run with the full warp
+            const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
+            if (!__all_sync(0xffffffffu, ok))
+                break;
+            tc_fence_after();
+            int mt, nt;
+            tile_coords(t, p, mt, nt);
+            const int m = mt * kBlockM + row;
+            const int n0 = nt * BN;
+            const bool m_ok = m < p.Mdim;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += C::EPI_CHUNK) {
+                uint32_t r[32];
+                tmem_ld_chunk<C::EPI_CHUNK>(taddr + c, r);
+                tmem_ld_wait();
+                if (m_ok) {
+                    OutT *o = out + static_cast<int64_t>(n0 + c) * p.ldo + m;
+#pragma unroll
+                    for (int j = 0; j < C::EPI_CHUNK; ++j)
+                        if (n0 + c + j < p.Ndim)
+                            store_out(o + static_cast<int64_t>(j) * p.ldo, r[j]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && *abort_flag && p.status)
+        atomicOr(p.status, 2);
+}
+
+}  // namespace lmh

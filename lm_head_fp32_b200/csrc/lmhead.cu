@@ -1,0 +1,317 @@
+// lmhead.cu -- C ABI of the LM-head loss path (declared in include/lmhead.h):
+// host-side argument validation, TMA descriptor encoding, kernel selection and
+// launch.  Every call only enqueues work on the caller's stream.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "lmhead.h"
+#include "ce_kernels.cuh"
+#include "gemm_tc.cuh"
+
+namespace {
+
+using lmh::GemmCfg;
+using lmh::GemmParams;
+
+constexpr int64_t kMaxDim = 0x7fffffff;
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int num_sms()
+{
+    static int cached[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// cuTensorMapEncodeTiled, resolved once through the runtime (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D BF16 tensor [outer, inner] (inner contiguous), 128-byte swizzled boxes
+// of box_inner x box_outer elements; out-of-range elements read as zero.
+bool make_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+lmh_status_t last_cuda_error()
+{
+    return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
+}
+
+// One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
+template <int BN, bool A_MN, bool B_MN, typename OutT>
+lmh_status_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, GemmParams p,
+                         cudaStream_t stream)
+{
+    using C = GemmCfg<BN, A_MN, B_MN>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT>;
+    // set once per process and device; the attribute is per function
+    static std::atomic<uint64_t> attr_set{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+            cudaSuccess)
+            return LMH_ERR_CUDA;
+        attr_set.fetch_or(bit);
+    }
+    p.num_m_tiles = static_cast<int32_t>((p.Mdim + lmh::kBlockM - 1) / lmh::kBlockM);
+    p.num_n_tiles = static_cast<int32_t>((p.Ndim + BN - 1) / BN);
+    const int64_t tiles = static_cast<int64_t>(p.num_m_tiles) * p.num_n_tiles;
+    if (tiles > kMaxDim)
+        return LMH_ERR_INVALID_ARG;
+    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+    kern<<<grid, lmh::kGemmThreads, C::SMEM_BYTES, stream>>>(ta, tb, p);
+    return last_cuda_error();
+}
+
+// Token-dimension tile width for the vocabulary GEMM and dX: the smallest
+// supported MMA N that covers M, capped at 256.
+int pick_bn_tokens(int64_t M)
+{
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+template <bool A_MN, bool B_MN, typename OutT>
+lmh_status_t dispatch_bn(int bn, const CUtensorMap &ta, const CUtensorMap &tb, GemmParams p,
+                         cudaStream_t s)
+{
+    if constexpr (!B_MN) {
+        switch (bn) {
+        case 16: return launch_gemm<16, A_MN, B_MN, OutT>(ta, tb, p, s);
+        case 32: return launch_gemm<32, A_MN, B_MN, OutT>(ta, tb, p, s);
+        default: break;
+        }
+    }
+    switch (bn) {
+    case 64: return launch_gemm<64, A_MN, B_MN, OutT>(ta, tb, p, s);
+    case 128: return launch_gemm<128, A_MN, B_MN, OutT>(ta, tb, p, s);
+    case 256: return launch_gemm<256, A_MN, B_MN, OutT>(ta, tb, p, s);
+    default: return LMH_ERR_UNSUPPORTED;
+    }
+}
+
+bool bad_dtype(int32_t t) { return t != LMH_F32 && t != LMH_BF16; }
+
+bool dims_ok(int64_t a, int64_t b, int64_t c)
+{
+    return a >= 1 && b >= 1 && c >= 1 && a <= kMaxDim && b <= kMaxDim && c <= kMaxDim;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lmh_status_string(lmh_status_t s)
+{
+    switch (s) {
+    case LMH_OK: return "ok";
+    case LMH_ERR_INVALID_ARG: return "invalid argument (null pointer or size out of range)";
+    case LMH_ERR_MISALIGNED: return "misaligned pointer or row stride";
+    case LMH_ERR_UNSUPPORTED: return "unsupported dtype or stride";
+    case LMH_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+int32_t lmh_version(void) { return 100; }
+
+lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_dtype, int64_t M,
+                        int64_t K, int64_t V, int32_t *status, lmh_stream_t stream)
+{
+    if (!X || !W || !logits || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (bad_dtype(out_dtype))
+        return LMH_ERR_UNSUPPORTED;
+    if (K % 8 || !aligned(X, 16) || !aligned(W, 16) ||
+        !aligned(logits, out_dtype == LMH_F32 ? 4 : 2))
+        return LMH_ERR_MISALIGNED;
+    const int bn = pick_bn_tokens(M);
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, W, K, V, lmh::kBlockK, lmh::kBlockM) || !make_map(&tb, X, K, M, lmh::kBlockK, bn))
+        return LMH_ERR_CUDA;
+    GemmParams p{};
+    p.out = logits;
+    p.ldo = V;
+    p.Mdim = static_cast<int32_t>(V);
+    p.Ndim = static_cast<int32_t>(M);
+    p.Kdim = static_cast<int32_t>(K);
+    p.m_fastest = 0;  // consecutive tiles share one W panel
+    p.status = status;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, ta, tb, p, s)
+                                : dispatch_bn<false, false, __nv_bfloat16>(bn, ta, tb, p, s);
+}
+
+lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t out_dtype,
+                           int64_t M, int64_t K, int64_t V, int32_t *status, lmh_stream_t stream)
+{
+    if (!dlogits || !W || !dX || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (bad_dtype(out_dtype))
+        return LMH_ERR_UNSUPPORTED;
+    if (K % 8 || V % 8 || !aligned(dlogits, 16) || !aligned(W, 16) ||
+        !aligned(dX, out_dtype == LMH_F32 ? 4 : 2))
+        return LMH_ERR_MISALIGNED;
+    const int bn = pick_bn_tokens(M);
+    CUtensorMap ta, tb;
+    // A = W^T (m = k_out contiguous, k = v), B = dl (n = token, k = v contiguous)
+    if (!make_map(&ta, W, K, V, 64, lmh::kBlockK) || !make_map(&tb, dlogits, V, M, lmh::kBlockK, bn))
+        return LMH_ERR_CUDA;
+    GemmParams p{};
+    p.out = dX;
+    p.ldo = K;
+    p.Mdim = static_cast<int32_t>(K);
+    p.Ndim = static_cast<int32_t>(M);
+    p.Kdim = static_cast<int32_t>(V);
+    p.m_fastest = 1;
+    p.status = status;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return out_dtype == LMH_F32 ? dispatch_bn<true, false, float>(bn, ta, tb, p, s)
+                                : dispatch_bn<true, false, __nv_bfloat16>(bn, ta, tb, p, s);
+}
+
+lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t out_dtype,
+                           int64_t M, int64_t K, int64_t V, int32_t *status, lmh_stream_t stream)
+{
+    if (!dlogits || !X || !dW || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (bad_dtype(out_dtype))
+        return LMH_ERR_UNSUPPORTED;
+    if (K % 8 || V % 8 || !aligned(dlogits, 16) || !aligned(X, 16) ||
+        !aligned(dW, out_dtype == LMH_F32 ? 4 : 2))
+        return LMH_ERR_MISALIGNED;
+    const int bn = V <= 64 ? 64 : V <= 128 ? 128 : 256;
+    CUtensorMap ta, tb;
+    // A = X^T (m = k_out contiguous, k = token), B = dl^T (n = v contiguous, k = token)
+    if (!make_map(&ta, X, K, M, 64, lmh::kBlockK) || !make_map(&tb, dlogits, V, M, 64, lmh::kBlockK))
+        return LMH_ERR_CUDA;
+    GemmParams p{};
+    p.out = dW;
+    p.ldo = K;
+    p.Mdim = static_cast<int32_t>(K);
+    p.Ndim = static_cast<int32_t>(V);
+    p.Kdim = static_cast<int32_t>(M);
+    p.m_fastest = 1;  // consecutive tiles share one dlogits panel
+    p.status = status;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return out_dtype == LMH_F32 ? dispatch_bn<true, true, float>(bn, ta, tb, p, s)
+                                : dispatch_bn<true, true, __nv_bfloat16>(bn, ta, tb, p, s);
+}
+
+lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, int64_t M, int64_t V,
+                    int64_t ignore_index, int32_t *status, lmh_stream_t stream)
+{
+    if (!logits || !target || !stats || M < 1 || V < 1 || M > kMaxDim || V > kMaxDim)
+        return LMH_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(target, 8) || !aligned(stats, 16))
+        return LMH_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+    const int grid = static_cast<int>(M < cap ? M : cap);
+    const bool vec = (V % 4 == 0) && aligned(logits, 16);
+    float4 *st4 = reinterpret_cast<float4 *>(stats);
+    if (vec)
+        lmh::ce_fwd_kernel<true><<<grid, lmh::kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
+    else
+        lmh::ce_fwd_kernel<false><<<grid, lmh::kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
+    return last_cuda_error();
+}
+
+lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *stats,
+                    const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
+                    int32_t dl_dtype, int64_t M, int64_t V, int64_t ignore_index,
+                    int32_t *status, lmh_stream_t stream)
+{
+    if (!logits || !target || !stats || !grad_loss || !dlogits || M < 1 || V < 1 ||
+        M > kMaxDim || V > kMaxDim)
+        return LMH_ERR_INVALID_ARG;
+    if (bad_dtype(dl_dtype) || (grad_loss_stride != 0 && grad_loss_stride != 1))
+        return LMH_ERR_UNSUPPORTED;
+    if (dl_dtype == LMH_BF16 && static_cast<const void *>(logits) == dlogits)
+        return LMH_ERR_UNSUPPORTED;  // in-place only for an FP32 gradient
+    if (!aligned(logits, 4) || !aligned(target, 8) || !aligned(stats, 16) || !aligned(grad_loss, 4) ||
+        !aligned(dlogits, dl_dtype == LMH_F32 ? 4 : 2))
+        return LMH_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+    const int grid = static_cast<int>(M < cap ? M : cap);
+    const float4 *st4 = reinterpret_cast<const float4 *>(stats);
+    if (dl_dtype == LMH_F32) {
+        float *o = static_cast<float *>(dlogits);
+        const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 16);
+        const bool alias = static_cast<const void *>(logits) == dlogits;
+        if (vec && alias)
+            lmh::ce_bwd_kernel<float, true, true><<<grid, lmh::kCeThreads, 0, s>>>(
+                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+        else if (vec)
+            lmh::ce_bwd_kernel<float, true, false><<<grid, lmh::kCeThreads, 0, s>>>(
+                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+        else if (alias)
+            lmh::ce_bwd_kernel<float, false, true><<<grid, lmh::kCeThreads, 0, s>>>(
+                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+        else
+            lmh::ce_bwd_kernel<float, false, false><<<grid, lmh::kCeThreads, 0, s>>>(
+                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+    } else {
+        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(dlogits);
+        const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 8);
+        if (vec)
+            lmh::ce_bwd_kernel<__nv_bfloat16, true, false><<<grid, lmh::kCeThreads, 0, s>>>(
+                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+        else
+            lmh::ce_bwd_kernel<__nv_bfloat16, false, false><<<grid, lmh::kCeThreads, 0, s>>>(
+                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+    }
+    return last_cuda_error();
+}
+
+}  // extern "C"

@@ -1,0 +1,156 @@
+"""ctypes binding of liblmhead.so: the five calls of include/lmhead.h.
+
+Argument marshalling only: shapes, dtypes and device pointers are read off
+torch tensors and passed to the C ABI on the caller's current CUDA stream.
+All arithmetic happens in the library's kernels.  If the library is missing
+or cannot be loaded, every call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblmhead.so")
+
+LMH_OK, LMH_ERR_INVALID_ARG, LMH_ERR_MISALIGNED, LMH_ERR_UNSUPPORTED, LMH_ERR_CUDA = range(5)
+F32, BF16, F16 = 0, 1, 2
+DEV_BAD_TARGET = 0x1
+DEV_PIPE_TIMEOUT = 0x2
+IGNORE_INDEX = -100
+
+EXPORTS = ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
+           "lmh_status_string", "lmh_version")
+
+_lib = None
+
+
+class LmhError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load liblmhead.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"liblmhead.so not found at {LIB_PATH}; build it with "
+                               "`python -m lm_head_fp32_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        L.lmhead_fwd.argtypes = [P, P, P, I32, I64, I64, I64, P, P]
+        L.ce_fwd.argtypes = [P, P, P, I64, I64, I64, P, P]
+        L.ce_bwd.argtypes = [P, P, P, P, I64, P, I32, I64, I64, I64, P, P]
+        L.lmhead_bwd_dx.argtypes = [P, P, P, I32, I64, I64, I64, P, P]
+        L.lmhead_bwd_dw.argtypes = [P, P, P, I32, I64, I64, I64, P, P]
+        for f in ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw"):
+            getattr(L, f).restype = ctypes.c_int
+        L.lmh_status_string.argtypes = [ctypes.c_int]
+        L.lmh_status_string.restype = ctypes.c_char_p
+        L.lmh_version.restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().lmh_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return F32
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float16:
+        return F16          # passed through so that the library rejects it
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _check(code: int, where: str):
+    if code != LMH_OK:
+        raise LmhError(code, where)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (row-major)")
+
+
+def lmhead_fwd(X: torch.Tensor, W: torch.Tensor, logits: torch.Tensor,
+               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """logits[M,V] (FP32 or BF16) = X[M,K] . W[V,K]^T."""
+    _contig(X, W, logits)
+    M, K = X.shape
+    V = W.shape[0]
+    assert W.shape[1] == K and tuple(logits.shape) == (M, V)
+    _check(lib().lmhead_fwd(_ptr(X), _ptr(W), _ptr(logits), _dtype_code(logits.dtype),
+                            M, K, V, _ptr(status), _stream(stream)), "lmhead_fwd")
+    return logits
+
+
+def ce_fwd(logits: torch.Tensor, target: torch.Tensor, stats: torch.Tensor,
+           ignore_index: int = IGNORE_INDEX, status: Optional[torch.Tensor] = None,
+           stream=None) -> torch.Tensor:
+    """stats[M,4] = {m, d, x_y, loss} per row of FP32 logits."""
+    _contig(logits, target, stats)
+    M, V = logits.shape
+    assert tuple(stats.shape) == (M, 4) and target.shape[0] == M
+    _check(lib().ce_fwd(_ptr(logits), _ptr(target), _ptr(stats), M, V, int(ignore_index),
+                        _ptr(status), _stream(stream)), "ce_fwd")
+    return stats
+
+
+def ce_bwd(logits: torch.Tensor, target: torch.Tensor, stats: torch.Tensor,
+           grad_loss: torch.Tensor, dlogits: torch.Tensor, ignore_index: int = IGNORE_INDEX,
+           status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dlogits = (softmax - onehot) * grad_loss in FP32, stored FP32 or BF16.
+    grad_loss: one element (broadcast to every row) or M elements."""
+    _contig(logits, target, stats, grad_loss, dlogits)
+    M, V = logits.shape
+    assert tuple(dlogits.shape) == (M, V)
+    stride = 0 if grad_loss.numel() == 1 else 1
+    if stride == 1:
+        assert grad_loss.numel() == M
+    _check(lib().ce_bwd(_ptr(logits), _ptr(target), _ptr(stats), _ptr(grad_loss), stride,
+                        _ptr(dlogits), _dtype_code(dlogits.dtype), M, V, int(ignore_index),
+                        _ptr(status), _stream(stream)), "ce_bwd")
+    return dlogits
+
+
+def lmhead_bwd_dx(dlogits: torch.Tensor, W: torch.Tensor, dX: torch.Tensor,
+                  status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dX[M,K] = dlogits[M,V] . W[V,K]."""
+    _contig(dlogits, W, dX)
+    M, V = dlogits.shape
+    K = W.shape[1]
+    assert W.shape[0] == V and tuple(dX.shape) == (M, K)
+    _check(lib().lmhead_bwd_dx(_ptr(dlogits), _ptr(W), _ptr(dX), _dtype_code(dX.dtype),
+                               M, K, V, _ptr(status), _stream(stream)), "lmhead_bwd_dx")
+    return dX
+
+
+def lmhead_bwd_dw(dlogits: torch.Tensor, X: torch.Tensor, dW: torch.Tensor,
+                  status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dW[V,K] = dlogits[M,V]^T . X[M,K]."""
+    _contig(dlogits, X, dW)
+    M, V = dlogits.shape
+    K = X.shape[1]
+    assert X.shape[0] == M and tuple(dW.shape) == (V, K)
+    _check(lib().lmhead_bwd_dw(_ptr(dlogits), _ptr(X), _ptr(dW), _dtype_code(dW.dtype),
+                               M, K, V, _ptr(status), _stream(stream)), "lmhead_bwd_dw")
+    return dW

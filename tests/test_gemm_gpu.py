@@ -1,0 +1,135 @@
+"""Parity of the three tcgen05 GEMMs (lmhead_fwd, lmhead_bwd_dx, lmhead_bwd_dw)
+with the FP64 oracle, through the C ABI.
+
+Integer-valued BF16 operands in [-8, 8] make every partial sum exact in FP32
+(Megatron-LM PR #6252, "Integer bitwise exactness results"), so those cases
+compare raw words; random operands use the K-scaled absolute tolerance."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lm_head_fp32_b200 import lmhead, synth
+from helpers import assert_abs_close, assert_bf16_close, bits, gemm_tol, logits_tol, to_f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def status_word():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+def gpu_logits(X, W, dtype=torch.float32):
+    M, V = X.shape[0], W.shape[0]
+    out = torch.empty((M, V), dtype=dtype, device=DEV)
+    st = status_word()
+    lmhead.lmhead_fwd(X.to(DEV), W.to(DEV), out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return out
+
+
+def gpu_dx(dl, W, dtype=torch.float32):
+    out = torch.empty((dl.shape[0], W.shape[1]), dtype=dtype, device=DEV)
+    st = status_word()
+    lmhead.lmhead_bwd_dx(dl.to(DEV), W.to(DEV), out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return out
+
+
+def gpu_dw(dl, X, dtype=torch.float32):
+    out = torch.empty((dl.shape[1], X.shape[1]), dtype=dtype, device=DEV)
+    st = status_word()
+    lmhead.lmhead_bwd_dw(dl.to(DEV), X.to(DEV), out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return out
+
+
+def test_integer_exactness_k_sweep(golden_dir):
+    """16 x K activations, 32768 x K weights, BF16 integers in [-8,8], seed 1234,
+    K in {512..16384}: the FP32 logits equal the exact result word for word."""
+    spec = json.load(open(os.path.join(golden_dir, "p1_integer_exactness.json")))
+    M, V = spec["activations_rows"], spec["vocab_rows"]
+    for K in spec["K"]:
+        X = synth.int_bf16((M, K), spec["seed"], spec["int_lo"], spec["int_hi"])
+        W = synth.int_bf16((V, K), spec["seed"] + 1, spec["int_lo"], spec["int_hi"])
+        out = gpu_logits(X, W)
+        ref = oracle.round_f32(oracle.logits(bits(X), bits(W)))
+        got = out.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), f"K={K}"
+        # the BF16 epilogue of the same kernel is the RNE of the same exact value
+        out16 = gpu_logits(X, W, torch.bfloat16)
+        ref16 = oracle.round_bf16(oracle.logits(bits(X), bits(W)))
+        assert np.array_equal(bits(out16), ref16), f"K={K} (BF16 epilogue)"
+
+
+@pytest.mark.parametrize("M,K,V", [(300, 1000, 1000), (17, 72, 32776), (130, 4096, 520),
+                                   (1, 8, 1), (257, 136, 129), (1024, 256, 384)])
+def test_logits_random_ragged(M, K, V):
+    X = synth.normal_bf16((M, K), 1.0, 11 + M)
+    W = synth.normal_bf16((V, K), 0.02, 12 + V)
+    ref = oracle.logits(bits(X), bits(W))
+    out = gpu_logits(X, W)
+    assert_abs_close(out.cpu().double().numpy(), ref, logits_tol(X, W), "FP32 logits")
+    out16 = gpu_logits(X, W, torch.bfloat16)
+    assert_bf16_close(out16, ref, "BF16 logits", abs_tol=logits_tol(X, W))
+
+
+def test_logits_deterministic():
+    X = synth.normal_bf16((512, 2048), 1.0, 1)
+    W = synth.normal_bf16((4096, 2048), 0.02, 2)
+    a = gpu_logits(X, W)
+    b = gpu_logits(X, W)
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("M,K,V", [(300, 264, 1000), (17, 72, 40), (1, 8, 8), (129, 520, 2056),
+                                   (1024, 128, 4096)])
+def test_grad_gemms_integer_exact(M, K, V):
+    dl = synth.int_bf16((M, V), 21 + M)
+    X = synth.int_bf16((M, K), 22 + K)
+    W = synth.int_bf16((V, K), 23 + V)
+    dX = gpu_dx(dl, W).cpu().numpy()
+    dW = gpu_dw(dl, X).cpu().numpy()
+    refx = oracle.round_f32(oracle.dx(bits(dl), bits(W)))
+    refw = oracle.round_f32(oracle.dw(bits(dl), bits(X)))
+    assert np.array_equal(dX.view(np.uint32), refx.view(np.uint32)), "dX"
+    assert np.array_equal(dW.view(np.uint32), refw.view(np.uint32)), "dW"
+
+
+@pytest.mark.parametrize("M,K,V", [(300, 264, 1000), (17, 4096, 32776), (200, 1000, 136)])
+def test_grad_gemms_random(M, K, V):
+    dl = synth.normal_bf16((M, V), 1e-3, 31 + M)
+    X = synth.normal_bf16((M, K), 1.0, 32 + K)
+    W = synth.normal_bf16((V, K), 0.02, 33 + V)
+    refx = oracle.dx(bits(dl), bits(W))
+    refw = oracle.dw(bits(dl), bits(X))
+    dX = gpu_dx(dl, W)
+    dW = gpu_dw(dl, X)
+    assert_abs_close(to_f64(dX), refx, gemm_tol(V, dl, W), "dX")
+    assert_abs_close(to_f64(dW), refw, gemm_tol(M, dl, X), "dW")
+    assert_bf16_close(gpu_dx(dl, W, torch.bfloat16), refx, "dX BF16", abs_tol=gemm_tol(V, dl, W))
+    assert_bf16_close(gpu_dw(dl, X, torch.bfloat16), refw, "dW BF16", abs_tol=gemm_tol(M, dl, X))
+    assert torch.equal(dX, gpu_dx(dl, W)) and torch.equal(dW, gpu_dw(dl, X))
+
+
+def test_grad_gemms_large_sampled():
+    """M=1024, K=4096, V=32768: sampled rows of dX and dW against the oracle."""
+    M, K, V = 1024, 4096, 32768
+    dl = synth.normal_bf16((M, V), 3e-5, 41)
+    X = synth.normal_bf16((M, K), 1.0, 42)
+    W = synth.normal_bf16((V, K), 0.02, 43)
+    dX, dW = gpu_dx(dl, W), gpu_dw(dl, X)
+    rng = np.random.default_rng(1239)
+    rx = np.sort(rng.choice(M, 12, replace=False))
+    rw = np.sort(np.concatenate([rng.choice(V, 24, replace=False), [0, V - 1]]))
+    assert_abs_close(to_f64(dX[torch.as_tensor(rx, device=DEV)]),
+                     oracle.dx(bits(dl), bits(W), rows=rx), gemm_tol(V, dl, W), "dX sampled")
+    assert_abs_close(to_f64(dW[torch.as_tensor(rw, device=DEV)]),
+                     oracle.dw(bits(dl), bits(X), vrows=rw), gemm_tol(M, dl, X), "dW sampled")
