@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-sample", type=int, default=96,
+    ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the workload the CPU oracle baseline processes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()

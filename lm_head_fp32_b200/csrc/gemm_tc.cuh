@@ -18,11 +18,16 @@
 // CTA roles (192 threads, one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: fills a STAGES-deep ring of A/B k-blocks
 //   warp 1      tensor-memory owner and MMA issuer (one elected thread)
-//   warps 2..5  epilogue: tensor memory -> registers -> global memory
+//   warps 2..5  epilogue: tensor memory -> registers -> shared memory -> TMA
+//               bulk tensor store (or, for outputs a tensor map cannot
+//               describe, registers -> global stores)
 // Two accumulators of BN columns let the epilogue of tile t overlap the MMAs
-// of tile t+1.  Every wait is bounded (see mbar_wait); on a timeout the CTA
-// drains its own copies and MMAs, frees tensor memory, sets a status bit and
-// returns.
+// of tile t+1.  With the TMA-store epilogue each warp stages 32 x 32 sub-tiles
+// in two shared-memory slots and hands them to the TMA engine, so tensor
+// memory is released as soon as its values are in shared memory instead of
+// after 128 KB of global stores have drained.  Every wait is bounded (see
+// mbar_wait); on a timeout the CTA drains its own copies and MMAs, frees
+// tensor memory, sets a status bit and returns.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -49,6 +54,9 @@ struct GemmParams {
     int32_t *status;
 };
 
+constexpr int kEpiWarps = 4;
+constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
+
 template <int BN, bool A_MN, bool B_MN>
 struct GemmCfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -56,15 +64,21 @@ struct GemmCfg {
     static constexpr int A_BYTES = kBlockM * kBlockK * 2;  // 16 KB
     static constexpr int B_BYTES = BN * kBlockK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
-    static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;
+    static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;  // accumulator columns per sub-tile
+    // two staging slots of 32 lanes x EPI_CHUNK columns per epilogue warp,
+    // sized for FP32 (a BF16 output uses half of each slot)
+    static constexpr int EPI_SLOT_BYTES = 32 * EPI_CHUNK * 4;
+    static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_SLOT_BYTES;
     // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
+    static constexpr int FIXED_BYTES = 1024 /* alignment slack */ + EPI_BYTES + 64 * 8;
+    static constexpr int STAGES_RAW = (kSmemLimit - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
-    static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + BAR_BYTES + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 16;
     static constexpr uint32_t IDESC = idesc_bf16_f32(kBlockM, BN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
     static_assert(STAGES >= 2, "pipeline depth");
+    static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
 };
 
 template <int N>
@@ -93,6 +107,11 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *p, uint32_t bits)
 {
     *p = __float2bfloat16_rn(__uint_as_float(bits));
 }
+__device__ __forceinline__ void stage_out(float *p, uint32_t bits) { *p = __uint_as_float(bits); }
+__device__ __forceinline__ void stage_out(__nv_bfloat16 *p, uint32_t bits)
+{
+    *p = __float2bfloat16_rn(__uint_as_float(bits));
+}
 
 __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt, int &nt)
 {
@@ -105,10 +124,12 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt,
     }
 }
 
-template <int BN, bool A_MN, bool B_MN, typename OutT>
+// TMA_STORE: the output is written through tmC, a tensor map over
+// out[Ndim][ldo] with box {32, EPI_CHUNK}; otherwise by direct global stores.
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p)
+                   const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
     using C = GemmCfg<BN, A_MN, B_MN>;
     constexpr int S = C::STAGES;
@@ -116,7 +137,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *tiles = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
+    uint8_t *epi_smem = smem + S * C::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(epi_smem + C::EPI_BYTES);
     uint64_t *full = bars;
     uint64_t *empty = bars + S;
     uint64_t *acc_full = bars + 2 * S;
@@ -144,6 +166,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (TMA_STORE)
+            tma_prefetch_desc(&tmC);
     }
     if (warp == 1)
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -256,6 +280,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int q = warp & 3;  // tensor-memory lane quarter this warp may access
         const int row = q * 32 + lane;
         OutT *out = static_cast<OutT *>(p.out);
+        OutT *slots = reinterpret_cast<OutT *>(epi_smem + (warp - 2) * 2 * C::EPI_SLOT_BYTES);
+        constexpr int SLOT_ELEMS = C::EPI_SLOT_BYTES / static_cast<int>(sizeof(float));
+        uint32_t slot = 0;
         uint32_t acc = 0, acc_phase = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             // every lane waits, then the warp agrees, so the .sync.aligned
@@ -272,10 +299,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
 #pragma unroll 1
             for (int c = 0; c < BN; c += C::EPI_CHUNK) {
+                if (TMA_STORE && n0 + c >= p.Ndim)
+                    break;  // the rest of this tile lies beyond the output
                 uint32_t r[32];
                 tmem_ld_chunk<C::EPI_CHUNK>(taddr + c, r);
                 tmem_ld_wait();
-                if (m_ok) {
+                if (TMA_STORE) {
+                    // slot is free once the store issued two sub-tiles ago
+                    // has finished reading it
+                    if (lane == 0)
+                        bulk_wait_read<1>();
+                    __syncwarp();
+                    OutT *buf = slots + slot * SLOT_ELEMS;
+#pragma unroll
+                    for (int j = 0; j < C::EPI_CHUNK; ++j)
+                        stage_out(buf + j * 32 + lane, r[j]);  // box row j = output row n0+c+j
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, buf, mt * kBlockM + q * 32, n0 + c);
+                        bulk_commit();
+                    }
+                    slot ^= 1;
+                } else if (m_ok) {
                     OutT *o = out + static_cast<int64_t>(n0 + c) * p.ldo + m;
 #pragma unroll
                     for (int j = 0; j < C::EPI_CHUNK; ++j)
@@ -290,6 +336,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 acc_phase ^= 1;
             }
         }
+        if (TMA_STORE && lane == 0)
+            bulk_wait_all();  // every output byte written before the CTA exits
     }
 
     tc_fence_before();

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "lmhead.h"
@@ -76,18 +77,40 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output tensor map for the TMA-store epilogue: [outer rows][row stride ld]
+// of FP32 or BF16, box {32, box_rows}, no swizzle.  False when the layout
+// cannot be described (base not 16-byte aligned, row stride not a multiple
+// of 16 bytes); the caller then uses the direct-store epilogue.
+bool make_out_map(CUtensorMap *map, void *base, bool bf16, uint64_t inner, uint64_t outer,
+                  uint64_t ld, uint32_t box_rows)
+{
+    const uint64_t esize = bf16 ? 2 : 4;
+    if (!aligned(base, 16) || (ld * esize) % 16 != 0)
+        return false;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {ld * esize};
+    const cuuint32_t box[2] = {32, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base,
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 lmh_status_t last_cuda_error()
 {
     return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
 
 // One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
-template <int BN, bool A_MN, bool B_MN, typename OutT>
-lmh_status_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, GemmParams p,
-                         cudaStream_t stream)
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE>
+lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
+                              GemmParams p, cudaStream_t stream)
 {
     using C = GemmCfg<BN, A_MN, B_MN>;
-    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -105,8 +128,21 @@ lmh_status_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, GemmParam
     if (tiles > kMaxDim)
         return LMH_ERR_INVALID_ARG;
     const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-    kern<<<grid, lmh::kGemmThreads, C::SMEM_BYTES, stream>>>(ta, tb, p);
+    kern<<<grid, lmh::kGemmThreads, C::SMEM_BYTES, stream>>>(ta, tb, tc, p);
     return last_cuda_error();
+}
+
+template <int BN, bool A_MN, bool B_MN, typename OutT>
+lmh_status_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, GemmParams p,
+                         cudaStream_t stream)
+{
+    using C = GemmCfg<BN, A_MN, B_MN>;
+    CUtensorMap tc;
+    if (make_out_map(&tc, p.out, sizeof(OutT) == 2, static_cast<uint64_t>(p.Mdim),
+                     static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
+        return launch_gemm_impl<BN, A_MN, B_MN, OutT, true>(ta, tb, tc, p, stream);
+    std::memset(&tc, 0, sizeof tc);
+    return launch_gemm_impl<BN, A_MN, B_MN, OutT, false>(ta, tb, tc, p, stream);
 }
 
 // Token-dimension tile width for the vocabulary GEMM and dX: the smallest

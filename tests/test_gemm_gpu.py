@@ -133,3 +133,30 @@ def test_grad_gemms_large_sampled():
                      oracle.dx(bits(dl), bits(W), rows=rx), gemm_tol(V, dl, W), "dX sampled")
     assert_abs_close(to_f64(dW[torch.as_tensor(rw, device=DEV)]),
                      oracle.dw(bits(dl), bits(X), vrows=rw), gemm_tol(M, dl, X), "dW sampled")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_direct_store_epilogue_on_unaligned_output(dtype):
+    """An output a tensor map cannot describe (base not 16-byte aligned) takes
+    the direct-store epilogue; the results are the same bits."""
+    M, K, V = 70, 264, 1000
+    X = synth.normal_bf16((M, K), 1.0, 5)
+    W = synth.normal_bf16((V, K), 0.02, 6)
+    dl = synth.normal_bf16((M, V), 1e-3, 7)
+    ref = gpu_logits(X, W, dtype)
+    refx, refw = gpu_dx(dl, W, dtype), gpu_dw(dl, X, dtype)
+    Xd, Wd, dld = X.to(DEV), W.to(DEV), dl.to(DEV)
+    for shape, fn, expect in [((M, V), lambda o, s: lmhead.lmhead_fwd(Xd, Wd, o, s), ref),
+                              ((M, K), lambda o, s: lmhead.lmhead_bwd_dx(dld, Wd, o, s), refx),
+                              ((V, K), lambda o, s: lmhead.lmhead_bwd_dw(dld, Xd, o, s), refw)]:
+        n = shape[0] * shape[1]
+        buf = torch.zeros(n + 8, dtype=dtype, device=DEV)
+        off = 1  # one element: 4 or 2 bytes past a 16-byte boundary
+        out = buf[off:off + n].view(shape)
+        assert out.data_ptr() % 16 != 0
+        st = status_word()
+        fn(out, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert torch.equal(out, expect)
+        assert bool((buf[:off] == 0).all()) and bool((buf[off + n:] == 0).all()), "wrote outside"
