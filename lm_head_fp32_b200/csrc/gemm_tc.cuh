@@ -57,13 +57,17 @@ struct GemmParams {
 constexpr int kEpiWarps = 4;
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, bool PAIR>
 struct GemmCfg {
+    static constexpr int CTAS = PAIR ? 2 : 1;
+    static constexpr int TILE_M = kBlockM * CTAS;  // m extent of one (pair) tile
+    static constexpr int BN_CTA = BN / CTAS;       // n rows of B held by each CTA
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-    static_assert(!B_MN || BN % 64 == 0, "MN-major B is loaded in 64-wide boxes");
+    static_assert(!PAIR || BN % 32 == 0, "pair MMA N");
+    static_assert(!B_MN || BN_CTA % 64 == 0, "MN-major B is loaded in 64-wide boxes");
     static constexpr int A_BYTES = kBlockM * kBlockK * 2;  // 16 KB
-    static constexpr int B_BYTES = BN * kBlockK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int B_BYTES = BN_CTA * kBlockK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
     static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;  // accumulator columns per sub-tile
     // two staging slots of 32 lanes x EPI_CHUNK columns per epilogue warp,
@@ -76,7 +80,7 @@ struct GemmCfg {
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 16;
-    static constexpr uint32_t IDESC = idesc_bf16_f32(kBlockM, BN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
+    static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
     static_assert(STAGES >= 2, "pipeline depth");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
 };
@@ -126,12 +130,17 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt,
 
 // TMA_STORE: the output is written through tmC, a tensor map over
 // out[Ndim][ldo] with box {32, EPI_CHUNK}; otherwise by direct global stores.
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE>
+// PAIR: a cluster of two CTAs on one tile of 256 (m) x BN (n) with
+// tcgen05.mma.cta_group::2 -- each CTA stages its own 128 rows of A and BN/2
+// rows of B, the leader (rank 0) issues the MMAs, and each CTA's tensor
+// memory receives its 128 rows of the accumulator.  B is read from L2 once
+// per pair instead of once per SM.
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using C = GemmCfg<BN, A_MN, B_MN>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -149,6 +158,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int num_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int num_tiles = p.num_m_tiles * p.num_n_tiles;
     const int num_kb = (p.Kdim + kBlockK - 1) / kBlockK;
 
@@ -159,7 +172,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4 * 32);
+            mbar_init(&acc_empty[a], kEpiWarps * C::CTAS);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -169,10 +182,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (TMA_STORE)
             tma_prefetch_desc(&tmC);
     }
-    if (warp == 1)
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR)
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        else
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+    }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync();  // the peer signals the leader's barriers only after they exist
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -184,10 +204,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t stage = 0, phase = 0;
             int64_t issued = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            for (int t = unit; t < num_tiles && ok; t += num_units) {
                 int mt, nt;
                 tile_coords(t, p, mt, nt);
-                const int m0 = mt * kBlockM, n0 = nt * BN;
+                const int m0 = mt * C::TILE_M + static_cast<int>(rank) * kBlockM;  // this CTA's A rows
+                const int nb0 = nt * BN + static_cast<int>(rank) * C::BN_CTA;     // this CTA's B rows
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
                         ok = false;
@@ -195,21 +216,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     uint8_t *sa = tiles + stage * C::STAGE_BYTES;
                     uint8_t *sb = sa + C::A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+                    // the leader's full barrier counts the bytes of both CTAs
+                    const uint32_t fb = PAIR ? mapa_shared(smem_u32(&full[stage]), 0) : 0u;
+                    if (leader)
+                        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES * C::CTAS);
                     const int k0 = kb * kBlockK;
                     if (A_MN) {
 #pragma unroll
-                        for (int j = 0; j < kBlockM / 64; ++j)
-                            tma_load_2d(&tmA, &full[stage], sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
+                        for (int j = 0; j < kBlockM / 64; ++j) {
+                            if (PAIR)
+                                tma_load_2d_pair(&tmA, fb, sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
+                            else
+                                tma_load_2d(&tmA, &full[stage], sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
+                        }
                     } else {
-                        tma_load_2d(&tmA, &full[stage], sa, k0, m0, pol_a);
+                        if (PAIR)
+                            tma_load_2d_pair(&tmA, fb, sa, k0, m0, pol_a);
+                        else
+                            tma_load_2d(&tmA, &full[stage], sa, k0, m0, pol_a);
                     }
                     if (B_MN) {
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(&tmB, &full[stage], sb + j * 64 * kBlockK * 2, n0 + 64 * j, k0, pol_b);
+                        for (int j = 0; j < C::BN_CTA / 64; ++j) {
+                            if (PAIR)
+                                tma_load_2d_pair(&tmB, fb, sb + j * 64 * kBlockK * 2, nb0 + 64 * j, k0, pol_b);
+                            else
+                                tma_load_2d(&tmB, &full[stage], sb + j * 64 * kBlockK * 2, nb0 + 64 * j, k0, pol_b);
+                        }
                     } else {
-                        tma_load_2d(&tmB, &full[stage], sb, k0, n0, pol_b);
+                        if (PAIR)
+                            tma_load_2d_pair(&tmB, fb, sb, k0, nb0, pol_b);
+                        else
+                            tma_load_2d(&tmB, &full[stage], sb, k0, nb0, pol_b);
                     }
                     ++issued;
                     if (++stage == S) {
@@ -220,18 +258,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             if (!ok) {
                 // let the copies already issued land before the CTA exits
-                volatile int no_abort = 0;
-                for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i)
-                    mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1), &no_abort);
+                if (PAIR) {
+                    sleep_ns(20000);  // the pair's barrier lives in the leader
+                } else {
+                    volatile int no_abort = 0;
+                    for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i)
+                        mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1), &no_abort,
+                                  kDrainLimitNs);
+                }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------ MMA issuer (pair: leader only)
+        if (lane == 0 && leader) {
             uint32_t stage = 0, phase = 0;
             uint32_t acc = 0, acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            for (int t = unit; t < num_tiles && ok; t += num_units) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) {
                     ok = false;
                     break;
@@ -254,9 +297,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                  : smem_desc_sw128(sa + k * 32, 16, 1024);
                         const uint64_t db = B_MN ? smem_desc_sw128(sb + k * 2048, 64 * kBlockK * 2, 1024)
                                                  : smem_desc_sw128(sb + k * 32, 16, 1024);
-                        mma_bf16(d_tmem, da, db, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                        if (PAIR)
+                            mma_bf16_pair(d_tmem, da, db, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                        else
+                            mma_bf16(d_tmem, da, db, C::IDESC, (kb | k) != 0 ? 1u : 0u);
                     }
-                    mma_commit(&empty[stage]);  // frees the smem slot when these MMAs finish
+                    // frees the smem slot (of both CTAs) when these MMAs finish
+                    if (PAIR)
+                        mma_commit_pair(&empty[stage], 0x3);
+                    else
+                        mma_commit(&empty[stage]);
                     if (++stage == S) {
                         stage = 0;
                         phase ^= 1;
@@ -264,16 +314,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 if (!ok)
                     break;
-                mma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+                // accumulator ready for the epilogue (of both CTAs)
+                if (PAIR)
+                    mma_commit_pair(&acc_full[acc], 0x3);
+                else
+                    mma_commit(&acc_full[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
             }
             // wait until every MMA issued by this thread has completed
-            mma_commit(drain);
+            if (PAIR)
+                mma_commit_pair(drain, 0x1);
+            else
+                mma_commit(drain);
             volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
+            mbar_wait(drain, 0, &no_abort, kDrainLimitNs);
         }
     } else {
         // ------------------------------------------------ epilogue (warps 2..5)
@@ -282,9 +339,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         OutT *out = static_cast<OutT *>(p.out);
         OutT *slots = reinterpret_cast<OutT *>(epi_smem + (warp - 2) * 2 * C::EPI_SLOT_BYTES);
         constexpr int SLOT_ELEMS = C::EPI_SLOT_BYTES / static_cast<int>(sizeof(float));
+        // where this warp releases an accumulator: the leader's barrier
+        const uint32_t empty_addr0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
         uint32_t slot = 0;
         uint32_t acc = 0, acc_phase = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        for (int t = unit; t < num_tiles; t += num_units) {
             // every lane waits, then the warp agrees, so the .sync.aligned
             // tensor-memory loads below always run with the full warp
             const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
@@ -293,7 +352,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             int mt, nt;
             tile_coords(t, p, mt, nt);
-            const int m = mt * kBlockM + row;
+            const int mbase = mt * C::TILE_M + static_cast<int>(rank) * kBlockM;
+            const int m = mbase + row;
             const int n0 = nt * BN;
             const bool m_ok = m < p.Mdim;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
@@ -317,7 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmC, buf, mt * kBlockM + q * 32, n0 + c);
+                        tma_store_2d(&tmC, buf, mbase + q * 32, n0 + c);
                         bulk_commit();
                     }
                     slot ^= 1;
@@ -330,7 +390,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
+            __syncwarp();
+            if (lane == 0) {
+                if (PAIR)
+                    mbar_arrive_cluster(empty_addr0 + acc * 8);
+                else
+                    mbar_arrive(&acc_empty[acc]);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1;
@@ -342,10 +408,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (PAIR) {
+        if (*abort_flag)
+            sleep_ns(20000);  // copies or arrivals of the peer still in flight
+        cluster_sync();       // both CTAs are done with tensor memory and barriers
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if (PAIR)
+            tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else
+            tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
     if (threadIdx.x == 0 && *abort_flag && p.status)
         atomicOr(p.status, 2);

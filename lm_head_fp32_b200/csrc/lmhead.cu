@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -104,13 +105,30 @@ lmh_status_t last_cuda_error()
     return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
 
+// A GEMM operand as a 2-D BF16 tensor [outer][inner] (inner contiguous).
+// mn_major: the inner dimension is the operand's m (or n) dimension and the
+// outer one its reduction dimension; otherwise the reverse.
+struct Operand {
+    const void *base;
+    uint64_t inner, outer;
+    bool mn_major;
+};
+
+// Tensor map of an operand for tiles of `rows` m/n rows x 64 k: K-major
+// operands are one box {64, rows}, MN-major ones boxes {64, 64}.
+bool make_operand_map(CUtensorMap *map, const Operand &op, uint32_t rows)
+{
+    return op.mn_major ? make_map(map, op.base, op.inner, op.outer, 64, lmh::kBlockK)
+                       : make_map(map, op.base, op.inner, op.outer, lmh::kBlockK, rows);
+}
+
 // One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE>
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR>
 lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                               GemmParams p, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, A_MN, B_MN>;
-    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -122,27 +140,46 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
             return LMH_ERR_CUDA;
         attr_set.fetch_or(bit);
     }
-    p.num_m_tiles = static_cast<int32_t>((p.Mdim + lmh::kBlockM - 1) / lmh::kBlockM);
+    p.num_m_tiles = static_cast<int32_t>((p.Mdim + C::TILE_M - 1) / C::TILE_M);
     p.num_n_tiles = static_cast<int32_t>((p.Ndim + BN - 1) / BN);
     const int64_t tiles = static_cast<int64_t>(p.num_m_tiles) * p.num_n_tiles;
     if (tiles > kMaxDim)
         return LMH_ERR_INVALID_ARG;
-    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-    kern<<<grid, lmh::kGemmThreads, C::SMEM_BYTES, stream>>>(ta, tb, tc, p);
+    const int64_t units = num_sms() / C::CTAS;  // CTAs (or CTA pairs) resident at once
+    const int grid = static_cast<int>((tiles < units ? tiles : units) * C::CTAS);
+    if (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid, 1, 1);
+        cfg.blockDim = dim3(lmh::kGemmThreads, 1, 1);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p) != cudaSuccess)
+            return LMH_ERR_CUDA;
+    } else {
+        kern<<<grid, lmh::kGemmThreads, C::SMEM_BYTES, stream>>>(ta, tb, tc, p);
+    }
     return last_cuda_error();
 }
 
-template <int BN, bool A_MN, bool B_MN, typename OutT>
-lmh_status_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, GemmParams p,
-                         cudaStream_t stream)
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool PAIR>
+lmh_status_t launch_gemm(const Operand &a, const Operand &b, GemmParams p, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, A_MN, B_MN>;
-    CUtensorMap tc;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
+    CUtensorMap ta, tb, tc;
+    if (!make_operand_map(&ta, a, lmh::kBlockM) || !make_operand_map(&tb, b, C::BN_CTA))
+        return LMH_ERR_CUDA;
     if (make_out_map(&tc, p.out, sizeof(OutT) == 2, static_cast<uint64_t>(p.Mdim),
                      static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
-        return launch_gemm_impl<BN, A_MN, B_MN, OutT, true>(ta, tb, tc, p, stream);
+        return launch_gemm_impl<BN, A_MN, B_MN, OutT, true, PAIR>(ta, tb, tc, p, stream);
     std::memset(&tc, 0, sizeof tc);
-    return launch_gemm_impl<BN, A_MN, B_MN, OutT, false>(ta, tb, tc, p, stream);
+    return launch_gemm_impl<BN, A_MN, B_MN, OutT, false, PAIR>(ta, tb, tc, p, stream);
 }
 
 // Token-dimension tile width for the vocabulary GEMM and dX: the smallest
@@ -156,21 +193,44 @@ int pick_bn_tokens(int64_t M)
     return 256;
 }
 
+// CTA-pair tiles (256 x 256) are used when the n extent fills a 256-wide
+// tile.  LMH_GEMM_PAIR=0 or 1 in the environment forces single-CTA or pair
+// tiles where both are possible (a tuning aid; read once per process).
+int pair_override()
+{
+    static int v = [] {
+        const char *e = std::getenv("LMH_GEMM_PAIR");
+        if (!e || !*e)
+            return -1;
+        return e[0] == '0' ? 0 : 1;
+    }();
+    return v;
+}
+
+bool use_pair(int bn, int64_t Mdim)
+{
+    if (bn != 256 || Mdim < 256)
+        return false;
+    const int o = pair_override();
+    return o < 0 ? true : o == 1;
+}
+
 template <bool A_MN, bool B_MN, typename OutT>
-lmh_status_t dispatch_bn(int bn, const CUtensorMap &ta, const CUtensorMap &tb, GemmParams p,
-                         cudaStream_t s)
+lmh_status_t dispatch_bn(int bn, const Operand &a, const Operand &b, GemmParams p, cudaStream_t s)
 {
     if constexpr (!B_MN) {
         switch (bn) {
-        case 16: return launch_gemm<16, A_MN, B_MN, OutT>(ta, tb, p, s);
-        case 32: return launch_gemm<32, A_MN, B_MN, OutT>(ta, tb, p, s);
+        case 16: return launch_gemm<16, A_MN, B_MN, OutT, false>(a, b, p, s);
+        case 32: return launch_gemm<32, A_MN, B_MN, OutT, false>(a, b, p, s);
         default: break;
         }
     }
     switch (bn) {
-    case 64: return launch_gemm<64, A_MN, B_MN, OutT>(ta, tb, p, s);
-    case 128: return launch_gemm<128, A_MN, B_MN, OutT>(ta, tb, p, s);
-    case 256: return launch_gemm<256, A_MN, B_MN, OutT>(ta, tb, p, s);
+    case 64: return launch_gemm<64, A_MN, B_MN, OutT, false>(a, b, p, s);
+    case 128: return launch_gemm<128, A_MN, B_MN, OutT, false>(a, b, p, s);
+    case 256:
+        return use_pair(bn, p.Mdim) ? launch_gemm<256, A_MN, B_MN, OutT, true>(a, b, p, s)
+                                    : launch_gemm<256, A_MN, B_MN, OutT, false>(a, b, p, s);
     default: return LMH_ERR_UNSUPPORTED;
     }
 }
@@ -211,9 +271,8 @@ lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_
         !aligned(logits, out_dtype == LMH_F32 ? 4 : 2))
         return LMH_ERR_MISALIGNED;
     const int bn = pick_bn_tokens(M);
-    CUtensorMap ta, tb;
-    if (!make_map(&ta, W, K, V, lmh::kBlockK, lmh::kBlockM) || !make_map(&tb, X, K, M, lmh::kBlockK, bn))
-        return LMH_ERR_CUDA;
+    const Operand a{W, static_cast<uint64_t>(K), static_cast<uint64_t>(V), false};  // A = W
+    const Operand b{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), false};  // B = X
     GemmParams p{};
     p.out = logits;
     p.ldo = V;
@@ -223,8 +282,8 @@ lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_
     p.m_fastest = 0;  // consecutive tiles share one W panel
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, ta, tb, p, s)
-                                : dispatch_bn<false, false, __nv_bfloat16>(bn, ta, tb, p, s);
+    return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, a, b, p, s)
+                                : dispatch_bn<false, false, __nv_bfloat16>(bn, a, b, p, s);
 }
 
 lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t out_dtype,
@@ -238,10 +297,9 @@ lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t
         !aligned(dX, out_dtype == LMH_F32 ? 4 : 2))
         return LMH_ERR_MISALIGNED;
     const int bn = pick_bn_tokens(M);
-    CUtensorMap ta, tb;
     // A = W^T (m = k_out contiguous, k = v), B = dl (n = token, k = v contiguous)
-    if (!make_map(&ta, W, K, V, 64, lmh::kBlockK) || !make_map(&tb, dlogits, V, M, lmh::kBlockK, bn))
-        return LMH_ERR_CUDA;
+    const Operand a{W, static_cast<uint64_t>(K), static_cast<uint64_t>(V), true};
+    const Operand b{dlogits, static_cast<uint64_t>(V), static_cast<uint64_t>(M), false};
     GemmParams p{};
     p.out = dX;
     p.ldo = K;
@@ -251,8 +309,8 @@ lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t
     p.m_fastest = 1;
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return out_dtype == LMH_F32 ? dispatch_bn<true, false, float>(bn, ta, tb, p, s)
-                                : dispatch_bn<true, false, __nv_bfloat16>(bn, ta, tb, p, s);
+    return out_dtype == LMH_F32 ? dispatch_bn<true, false, float>(bn, a, b, p, s)
+                                : dispatch_bn<true, false, __nv_bfloat16>(bn, a, b, p, s);
 }
 
 lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t out_dtype,
@@ -266,10 +324,9 @@ lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t
         !aligned(dW, out_dtype == LMH_F32 ? 4 : 2))
         return LMH_ERR_MISALIGNED;
     const int bn = V <= 64 ? 64 : V <= 128 ? 128 : 256;
-    CUtensorMap ta, tb;
     // A = X^T (m = k_out contiguous, k = token), B = dl^T (n = v contiguous, k = token)
-    if (!make_map(&ta, X, K, M, 64, lmh::kBlockK) || !make_map(&tb, dlogits, V, M, 64, lmh::kBlockK))
-        return LMH_ERR_CUDA;
+    const Operand a{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), true};
+    const Operand b{dlogits, static_cast<uint64_t>(V), static_cast<uint64_t>(M), true};
     GemmParams p{};
     p.out = dW;
     p.ldo = K;
@@ -279,8 +336,8 @@ lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t
     p.m_fastest = 1;  // consecutive tiles share one dlogits panel
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return out_dtype == LMH_F32 ? dispatch_bn<true, true, float>(bn, ta, tb, p, s)
-                                : dispatch_bn<true, true, __nv_bfloat16>(bn, ta, tb, p, s);
+    return out_dtype == LMH_F32 ? dispatch_bn<true, true, float>(bn, a, b, p, s)
+                                : dispatch_bn<true, true, __nv_bfloat16>(bn, a, b, p, s);
 }
 
 lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, int64_t M, int64_t V,
