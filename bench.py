@@ -5,6 +5,13 @@ on one synthetic batch (M=1024 tokens, K=4096, V=32768; X ~ N(0,1),
 W ~ N(0,0.02^2) in BF16, 2% of targets ignored, grad_loss = 1/num_valid).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload lmhead_1024x4096x32768 | lmhead_4096x4096x128256 |
+                                ce_8192x151936_outliers | sweep]
+
+The default workload is the one the metric is quoted on.  The other LM-head
+workload and the wide-row cross-entropy workload print the same kind of line;
+"sweep" runs the FP32-versus-BF16 output comparison of the GEMM (15 shapes,
+N = 32768, 10 warm-up pairs, 30 alternating-order samples, medians).
 
 Prints one JSON line on rank 0.  Timing: CUDA events on the launching stream
 around every step (and every call inside it), L2 flushed by a 512 MiB write
@@ -51,6 +58,9 @@ def parse():
     ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the workload the CPU oracle baseline processes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="lmhead_1024x4096x32768",
+                    choices=["lmhead_1024x4096x32768", "lmhead_4096x4096x128256",
+                             "ce_8192x151936_outliers", "sweep"])
     return ap.parse_args()
 
 
@@ -239,16 +249,21 @@ def run_reference(args):
 # GPU arm
 # ----------------------------------------------------------------------------
 
-def run_ours(args):
+def gpu_setup(args):
     import torch
-    from lm_head_fp32_b200 import lmhead, synth
-
     world, rank, local, pg = dist_setup(args)
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = synth.MIDSIZE
+    return world, rank, local, pg, dev
+
+
+def run_ours(args, cfg):
+    import torch
+    from lm_head_fp32_b200 import lmhead, synth
+
+    world, rank, local, pg, dev = gpu_setup(args)
     M, K, V = cfg.M, cfg.K, cfg.V
     # every rank draws its own batch (replica r uses seed + 7919 r)
     rcfg = synth.GemmConfig(cfg.name, M, K, V, cfg.dist, cfg.x_std, cfg.w_std, cfg.ignore_frac,
@@ -376,7 +391,160 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": len(calls) * K_steps, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, X, W, t, g, args.cpu_sample)
+        # about 10-30 s of oracle work: the sample shrinks as the vocabulary grows
+        sample = max(8, int(args.cpu_sample * 32768 * 4096 / (cfg.V * cfg.K)))
+        line["cpu_baseline"] = cpu_baseline(cfg, X, W, t, g, sample)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def run_ce(args):
+    """Wide-row cross-entropy workload: CE forward, CE backward with FP32
+    dlogits, CE backward with BF16 dlogits (g = 1)."""
+    import numpy as np
+    import torch
+    from lm_head_fp32_b200 import lmhead, synth
+
+    world, rank, local, pg, dev = gpu_setup(args)
+    cfg = synth.CE_WIDE
+    R, Cc = cfg.rows, cfg.cols
+    x, t, _ = cfg.make(device=dev)
+    td = t.to(dev)
+    st = torch.empty((R, 4), dtype=torch.float32, device=dev)
+    g = torch.ones(1, dtype=torch.float32, device=dev)
+    d32 = torch.empty((R, Cc), dtype=torch.float32, device=dev)
+    d16 = torch.empty((R, Cc), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["ce_fwd", "ce_bwd_f32", "ce_bwd_bf16"]
+    calls = [lambda: lmhead.ce_fwd(x, td, st, -100, status),
+             lambda: lmhead.ce_bwd(x, td, st, g, d32, -100, status),
+             lambda: lmhead.ce_bwd(x, td, st, g, d16, -100, status)]
+    for _ in range(max(args.warmup, 3)):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    steps = min(args.steps, 30)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(pg)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)
+    for i in range(steps):
+        e = ev[i]
+        e[0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            e[j + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(pg)
+    assert int(status.item()) == 0
+    total_ms = max_over_ranks(sum(ev[i][0].elapsed_time(ev[i][-1]) for i in range(steps)), pg, dev)
+    peaks, peak_src = load_peaks()
+    nv = int((t != -100).sum())
+    algo = {"ce_fwd": nv * Cc * 4 + R * 24, "ce_bwd_f32": nv * Cc * 4 + R * Cc * 4 + R * 24,
+            "ce_bwd_bf16": nv * Cc * 4 + R * Cc * 2 + R * 24}
+    kernels = {}
+    for j, n in enumerate(names):
+        ms = statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps))
+        gbs = algo[n] / (ms / 1e3) / 1e9
+        kernels[n] = {"ms": round(ms, 5), "bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s",
+                      "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic": algo[n]}
+    dom = max(names, key=lambda n: kernels[n]["ms"])
+    line = {"metric": METRIC, "value": world * R * steps / (total_ms / 1e3), "unit": "rows/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": cfg.name, "rows": R, "cols": Cc, "ignored_rows": R - nv,
+                       "outlier_rows": int(cfg.outlier_frac * R), "grad_loss": 1.0,
+                       "l2": "inputs (5 GB) larger than L2"},
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["achieved"],
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kernels[dom]["frac"],
+                         "peak_source": f"{peak_src} (copy)", "traffic": committed_traffic().get(dom)},
+            "kernels": kernels, "gpu_launches": len(calls) * steps, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        rows = np.arange(512, dtype=np.int64)
+        xs = x[:512].cpu().numpy()
+        ts = t.numpy()[:512]
+        t0 = time.perf_counter()
+        oracle.ce_fwd(xs, ts)
+        oracle.ce_bwd(xs, ts, 1.0)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": len(rows) / dt, "unit": "rows/s",
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"512 of {R} rows, CE forward + backward, FP64, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def run_sweep(args):
+    """FP32- versus BF16-output epilogue of the same GEMM over the 15 shapes
+    M x K (N = 32768): 10 warm-up pairs, 30 alternating-order event-timed
+    samples per kernel, medians (the protocol of the pages' GEMM benchmark)."""
+    import torch
+    from lm_head_fp32_b200 import lmhead, synth
+
+    world, rank, local, pg, dev = gpu_setup(args)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    peaks, peak_src = load_peaks()
+    rows = []
+    for c in synth.sweep_configs():
+        X = synth.normal_bf16((c.M, c.K), 1.0, c.seed, device=dev)
+        W = synth.normal_bf16((c.V, c.K), 0.02, c.seed + 1, device=dev)
+        o32 = torch.empty((c.M, c.V), dtype=torch.float32, device=dev)
+        o16 = torch.empty((c.M, c.V), dtype=torch.bfloat16, device=dev)
+        run = {"f32": lambda: lmhead.lmhead_fwd(X, W, o32, status),
+               "bf16": lambda: lmhead.lmhead_fwd(X, W, o16, status)}
+
+        def sample(k):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run[k]()
+            b.record(stream)
+            b.synchronize()
+            return a.elapsed_time(b)
+
+        for _ in range(10):
+            sample("f32")
+            sample("bf16")
+        t = {"f32": [], "bf16": []}
+        for i in range(30):
+            order = ("f32", "bf16") if i % 2 == 0 else ("bf16", "f32")
+            for k in order:
+                t[k].append(sample(k))
+        m32, m16 = statistics.median(t["f32"]), statistics.median(t["bf16"])
+        flop = 2.0 * c.M * c.K * c.V
+        bytes32 = 2.0 * c.V * c.K + 2.0 * c.M * c.K + 4.0 * c.M * c.V
+        bound = "hbm" if c.M <= 128 else "tensor"
+        ach = (bytes32 / (m32 / 1e3) / 1e9) if bound == "hbm" else (flop / (m32 / 1e3) / 1e12)
+        peak = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"]
+        rows.append({"M": c.M, "K": c.K, "N": c.V, "f32_us": round(m32 * 1e3, 2),
+                     "bf16_us": round(m16 * 1e3, 2),
+                     "overhead_pct": round(100.0 * (m32 - m16) / m16, 2),
+                     "f32_tflops": round(flop / (m32 / 1e3) / 1e12, 1), "bound": bound,
+                     "f32_frac": round(ach / peak, 4)})
+        del X, W, o32, o16
+    assert int(status.item()) == 0
+    ov = [r["overhead_pct"] for r in rows]
+    ov4 = [r["overhead_pct"] for r in rows if r["K"] >= 4096]
+    ov8 = [r["overhead_pct"] for r in rows if r["K"] >= 8192]
+    line = {"metric": "FP32-output vs BF16-output GEMM overhead, same kernel", "unit": "%",
+            "value": statistics.median(ov), "higher_is_better": False, "n_gpus": 1,
+            "median_overhead_pct_K_ge_4096": statistics.median(ov4),
+            "median_overhead_pct_K_ge_8192": statistics.median(ov8),
+            "shapes_within_10pct": sum(1 for o in ov if o <= 10.0),
+            "range_pct": [min(ov), max(ov)], "shapes": rows, "peak_source": peak_src,
+            "protocol": "10 warm-up pairs, 30 alternating-order samples, medians, L2 flushed"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -387,8 +555,16 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    from lm_head_fp32_b200 import synth
+    if args.workload == "sweep":
+        run_sweep(args)
+    elif args.workload == "ce_8192x151936_outliers":
+        run_ce(args)
+    elif args.workload == "lmhead_4096x4096x128256":
+        run_ours(args, synth.LARGEVOCAB)
     else:
-        run_ours(args)
+        run_ours(args, synth.MIDSIZE)
 
 
 if __name__ == "__main__":

@@ -6,16 +6,16 @@
 // writing gradients; the backward recomputes softmax from the saved (m, d) in
 // FP32 and writes the gradient, so each kernel reads the logits once.
 //
-// Both kernels are HBM-bound row sweeps: one CTA per row (grid-stride over
-// rows), 128-bit read-only streaming loads, an online (max, sum-exp) pair per
-// thread merged by warp shuffles and then across warps in shared memory.
+// Both kernels are HBM-bound row sweeps: one CTA per row (the loops also
+// stride over rows, so any grid works), 128-bit read-only streaming loads, an
+// online (max, sum-exp) pair per thread merged by warp shuffles and then
+// across warps in shared memory.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
 
 namespace lmh {
 
-constexpr int kCeThreads = 512;
 constexpr float kLog2e = 1.4426950408889634f;  // 1 / ln 2
 
 struct MaxSum {
@@ -134,8 +134,8 @@ __device__ __forceinline__ int row_kind(int64_t y, int64_t V, int64_t ignore_ind
 }
 
 // stats[row] = {m, d, x_y, loss}.  VEC: V % 4 == 0 and logits 16-byte aligned.
-template <bool VEC>
-__global__ void __launch_bounds__(kCeThreads) ce_fwd_kernel(const float *__restrict__ logits,
+template <bool VEC, int THREADS = 512>
+__global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict__ logits,
                                                             const int64_t *__restrict__ target,
                                                             float4 *__restrict__ stats, int64_t M,
                                                             int64_t V, int64_t ignore_index,
@@ -160,21 +160,21 @@ __global__ void __launch_bounds__(kCeThreads) ce_fwd_kernel(const float *__restr
             const int64_t n4 = V >> 2;
             int64_t i = threadIdx.x;
             // four 128-bit loads in flight per thread per step
-            for (; i + 3 * kCeThreads < n4; i += 4 * kCeThreads) {
-                float4 a = ldg_stream(x4 + i), b = ldg_stream(x4 + i + kCeThreads),
-                       c = ldg_stream(x4 + i + 2 * kCeThreads),
-                       e = ldg_stream(x4 + i + 3 * kCeThreads);
+            for (; i + 3 * THREADS < n4; i += 4 * THREADS) {
+                float4 a = ldg_stream(x4 + i), b = ldg_stream(x4 + i + THREADS),
+                       c = ldg_stream(x4 + i + 2 * THREADS),
+                       e = ldg_stream(x4 + i + 3 * THREADS);
                 const float v[16] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w,
                                      c.x, c.y, c.z, c.w, e.x, e.y, e.z, e.w};
                 fold<16>(s, v);
             }
-            for (; i < n4; i += kCeThreads) {
+            for (; i < n4; i += THREADS) {
                 float4 a = ldg_stream(x4 + i);
                 const float v[4] = {a.x, a.y, a.z, a.w};
                 fold<4>(s, v);
             }
         } else {
-            for (int64_t j = threadIdx.x; j < V; j += kCeThreads)
+            for (int64_t j = threadIdx.x; j < V; j += THREADS)
                 fold1(s, ldg_stream1(x + j));
         }
         s = block_merge(s, red);
@@ -217,8 +217,8 @@ __device__ __forceinline__ void store1(__nv_bfloat16 *p, float a) { *p = __float
 // Each element is read before it is written, by the same thread, so dl may
 // alias logits when OutT is float (ALIAS: coherent loads instead of the
 // read-only path).
-template <typename OutT, bool VEC, bool ALIAS>
-__global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(
+template <typename OutT, bool VEC, bool ALIAS, int THREADS = 512>
+__global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
     const float *logits, const int64_t *__restrict__ target, const float4 *__restrict__ stats,
     const float *__restrict__ grad_loss, int64_t grad_stride, OutT *dl, int64_t M, int64_t V,
     int64_t ignore_index, int32_t *status)
@@ -232,10 +232,10 @@ __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(
             if (kind == 2 && status && threadIdx.x == 0)
                 atomicOr(status, 1);
             if (VEC) {
-                for (int64_t i = threadIdx.x; i < (V >> 2); i += kCeThreads)
+                for (int64_t i = threadIdx.x; i < (V >> 2); i += THREADS)
                     store4<OutT>(o + 4 * i, 0.f, 0.f, 0.f, 0.f);
             } else {
-                for (int64_t j = threadIdx.x; j < V; j += kCeThreads)
+                for (int64_t j = threadIdx.x; j < V; j += THREADS)
                     store1(o + j, 0.f);
             }
             continue;
@@ -248,9 +248,9 @@ __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
             const int64_t n4 = V >> 2;
             int64_t i = threadIdx.x;
-            for (; i + kCeThreads < n4; i += 2 * kCeThreads) {
-                const float4 a = load4<ALIAS>(x4 + i), b = load4<ALIAS>(x4 + i + kCeThreads);
-                const int64_t ja = 4 * i, jb = 4 * (i + kCeThreads);
+            for (; i + THREADS < n4; i += 2 * THREADS) {
+                const float4 a = load4<ALIAS>(x4 + i), b = load4<ALIAS>(x4 + i + THREADS);
+                const int64_t ja = 4 * i, jb = 4 * (i + THREADS);
                 store4<OutT>(o + ja, (exp_neg(a.x - m) * inv_d - (ja + 0 == y)) * g,
                              (exp_neg(a.y - m) * inv_d - (ja + 1 == y)) * g,
                              (exp_neg(a.z - m) * inv_d - (ja + 2 == y)) * g,
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(
                              (exp_neg(b.z - m) * inv_d - (jb + 2 == y)) * g,
                              (exp_neg(b.w - m) * inv_d - (jb + 3 == y)) * g);
             }
-            for (; i < n4; i += kCeThreads) {
+            for (; i < n4; i += THREADS) {
                 const float4 a = load4<ALIAS>(x4 + i);
                 const int64_t ja = 4 * i;
                 store4<OutT>(o + ja, (exp_neg(a.x - m) * inv_d - (ja + 0 == y)) * g,
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kCeThreads) ce_bwd_kernel(
                              (exp_neg(a.w - m) * inv_d - (ja + 3 == y)) * g);
             }
         } else {
-            for (int64_t j = threadIdx.x; j < V; j += kCeThreads) {
+            for (int64_t j = threadIdx.x; j < V; j += THREADS) {
                 const float v = load1<ALIAS>(x + j);
                 store1(o + j, (exp_neg(v - m) * inv_d - (j == y)) * g);
             }

@@ -22,6 +22,7 @@ using lmh::GemmParams;
 
 constexpr int64_t kMaxDim = 0x7fffffff;
 constexpr int kMaxDevices = 64;
+constexpr int kCeThreads = 1024;  // threads per cross-entropy CTA; one CTA per row
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -348,14 +349,14 @@ lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, in
     if (!aligned(logits, 4) || !aligned(target, 8) || !aligned(stats, 16))
         return LMH_ERR_MISALIGNED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
-    const int grid = static_cast<int>(M < cap ? M : cap);
+    // one CTA per row: the block scheduler balances rows across SMs
+    const int grid = static_cast<int>(M);
     const bool vec = (V % 4 == 0) && aligned(logits, 16);
     float4 *st4 = reinterpret_cast<float4 *>(stats);
     if (vec)
-        lmh::ce_fwd_kernel<true><<<grid, lmh::kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
+        lmh::ce_fwd_kernel<true, kCeThreads><<<grid, kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
     else
-        lmh::ce_fwd_kernel<false><<<grid, lmh::kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
+        lmh::ce_fwd_kernel<false, kCeThreads><<<grid, kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
     return last_cuda_error();
 }
 
@@ -375,33 +376,33 @@ lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *sta
         !aligned(dlogits, dl_dtype == LMH_F32 ? 4 : 2))
         return LMH_ERR_MISALIGNED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
-    const int grid = static_cast<int>(M < cap ? M : cap);
+    // one CTA per row: the block scheduler balances rows across SMs
+    const int grid = static_cast<int>(M);
     const float4 *st4 = reinterpret_cast<const float4 *>(stats);
     if (dl_dtype == LMH_F32) {
         float *o = static_cast<float *>(dlogits);
         const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 16);
         const bool alias = static_cast<const void *>(logits) == dlogits;
         if (vec && alias)
-            lmh::ce_bwd_kernel<float, true, true><<<grid, lmh::kCeThreads, 0, s>>>(
+            lmh::ce_bwd_kernel<float, true, true, kCeThreads><<<grid, kCeThreads, 0, s>>>(
                 logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
         else if (vec)
-            lmh::ce_bwd_kernel<float, true, false><<<grid, lmh::kCeThreads, 0, s>>>(
+            lmh::ce_bwd_kernel<float, true, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
                 logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
         else if (alias)
-            lmh::ce_bwd_kernel<float, false, true><<<grid, lmh::kCeThreads, 0, s>>>(
+            lmh::ce_bwd_kernel<float, false, true, kCeThreads><<<grid, kCeThreads, 0, s>>>(
                 logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
         else
-            lmh::ce_bwd_kernel<float, false, false><<<grid, lmh::kCeThreads, 0, s>>>(
+            lmh::ce_bwd_kernel<float, false, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
                 logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
     } else {
         __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(dlogits);
         const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 8);
         if (vec)
-            lmh::ce_bwd_kernel<__nv_bfloat16, true, false><<<grid, lmh::kCeThreads, 0, s>>>(
+            lmh::ce_bwd_kernel<__nv_bfloat16, true, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
                 logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
         else
-            lmh::ce_bwd_kernel<__nv_bfloat16, false, false><<<grid, lmh::kCeThreads, 0, s>>>(
+            lmh::ce_bwd_kernel<__nv_bfloat16, false, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
                 logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
     }
     return last_cuda_error();
