@@ -323,32 +323,51 @@ def run_ours(args, cfg):
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     value = world * M * K_steps / (total_ms / 1e3)
 
-    # end to end through the public API: pinned host X and targets in, loss out
+    # end to end through the public API: every step copies its X and targets
+    # from pinned host memory and reads its per-row loss back.  Inputs are
+    # double-buffered and copied on a second stream, so step i+1's copy runs
+    # under step i's kernels, as in a training loop with a prefetching loader.
     Xh = X.pin_memory()
     th = t.pin_memory()
-    lossh = torch.empty((M, 4), dtype=torch.float32).pin_memory()
-    e2e_steps = max(10, min(K_steps, 50))
-    for _ in range(3):
-        Xd.copy_(Xh, non_blocking=True)
-        td.copy_(th, non_blocking=True)
-        step()
-        lossh.copy_(stats, non_blocking=True)
+    lossh = [torch.empty((M, 4), dtype=torch.float32).pin_memory() for _ in range(2)]
+    Xb = [Xd, torch.empty_like(Xd)]
+    tb = [td, torch.empty_like(td)]
+    cs = torch.cuda.Stream(device=dev)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(i):
+        b = i % 2
+        if i >= 2:
+            cs.wait_event(done[b])          # step i-2 has finished with buffer b
+        with torch.cuda.stream(cs):
+            Xb[b].copy_(Xh, non_blocking=True)
+            tb[b].copy_(th, non_blocking=True)
+            copied[b].record(cs)
+        stream.wait_event(copied[b])
+        lmhead.lmhead_fwd(Xb[b], Wd, logits, status)
+        lmhead.ce_fwd(logits, tb[b], stats, -100, status)
+        lmhead.ce_bwd(logits, tb[b], stats, gd, dl, -100, status)
+        lmhead.lmhead_bwd_dx(dl, Wd, dX, status)
+        lmhead.lmhead_bwd_dw(dl, Xb[b], dW, status)
+        lossh[b].copy_(stats, non_blocking=True)
+        done[b].record(stream)
+
+    e2e_steps = max(10, min(K_steps, 100))
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize()
-    e2e_ms = 0.0
-    for _ in range(e2e_steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        Xd.copy_(Xh, non_blocking=True)
-        td.copy_(th, non_blocking=True)
-        step()
-        lossh.copy_(stats, non_blocking=True)
-        b.record(stream)
-        b.synchronize()
-        e2e_ms += a.elapsed_time(b)
-    e2e_ms = max_over_ranks(e2e_ms, pg, dev)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    cs.wait_event(a)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    z.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(z), pg, dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
     h2d = Xh.numel() * Xh.element_size() + th.numel() * th.element_size()
-    d2h = lossh.numel() * lossh.element_size()
+    d2h = lossh[0].numel() * lossh[0].element_size()
 
     # roofline of every kernel; the dominant one goes in "roofline"
     peaks, peak_src = load_peaks()
@@ -388,7 +407,9 @@ def run_ours(args, cfg):
                        "parallelism": f"replicas x{world}"},
             "roofline": roofline, "kernels": kernels,
             "e2e": {"value": world * M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "note": "pinned-host inputs copied on a second stream, double-buffered; "
+                            "no L2 flush (the step's working set is far larger than L2)"},
             "gpu_launches": len(calls) * K_steps, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of oracle work: the sample shrinks as the vocabulary grows

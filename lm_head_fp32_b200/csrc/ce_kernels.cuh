@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
             const int64_t n4 = V >> 2;
             int64_t i = threadIdx.x;
-            // four 128-bit loads in flight per thread per step
+            // four independent 128-bit loads in flight per thread per step
             for (; i + 3 * THREADS < n4; i += 4 * THREADS) {
                 float4 a = ldg_stream(x4 + i), b = ldg_stream(x4 + i + THREADS),
                        c = ldg_stream(x4 + i + 2 * THREADS),
@@ -223,7 +223,10 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
     const float *__restrict__ grad_loss, int64_t grad_stride, OutT *dl, int64_t M, int64_t V,
     int64_t ignore_index, int32_t *status)
 {
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    // rows in the opposite order to ce_fwd: the rows it read last are the
+    // ones most likely still in L2
+    for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
+        const int64_t row = M - 1 - r;
         const int64_t y = target[row];
         const int kind = row_kind(y, V, ignore_index);
         const float *x = logits + row * V;
@@ -248,17 +251,20 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
             const int64_t n4 = V >> 2;
             int64_t i = threadIdx.x;
-            for (; i + THREADS < n4; i += 2 * THREADS) {
-                const float4 a = load4<ALIAS>(x4 + i), b = load4<ALIAS>(x4 + i + THREADS);
-                const int64_t ja = 4 * i, jb = 4 * (i + THREADS);
-                store4<OutT>(o + ja, (exp_neg(a.x - m) * inv_d - (ja + 0 == y)) * g,
-                             (exp_neg(a.y - m) * inv_d - (ja + 1 == y)) * g,
-                             (exp_neg(a.z - m) * inv_d - (ja + 2 == y)) * g,
-                             (exp_neg(a.w - m) * inv_d - (ja + 3 == y)) * g);
-                store4<OutT>(o + jb, (exp_neg(b.x - m) * inv_d - (jb + 0 == y)) * g,
-                             (exp_neg(b.y - m) * inv_d - (jb + 1 == y)) * g,
-                             (exp_neg(b.z - m) * inv_d - (jb + 2 == y)) * g,
-                             (exp_neg(b.w - m) * inv_d - (jb + 3 == y)) * g);
+            // four independent 128-bit loads in flight per thread per step
+            for (; i + 3 * THREADS < n4; i += 4 * THREADS) {
+                float4 a[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    a[u] = load4<ALIAS>(x4 + i + u * THREADS);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t ja = 4 * (i + u * THREADS);
+                    store4<OutT>(o + ja, (exp_neg(a[u].x - m) * inv_d - (ja + 0 == y)) * g,
+                                 (exp_neg(a[u].y - m) * inv_d - (ja + 1 == y)) * g,
+                                 (exp_neg(a[u].z - m) * inv_d - (ja + 2 == y)) * g,
+                                 (exp_neg(a[u].w - m) * inv_d - (ja + 3 == y)) * g);
+                }
             }
             for (; i < n4; i += THREADS) {
                 const float4 a = load4<ALIAS>(x4 + i);

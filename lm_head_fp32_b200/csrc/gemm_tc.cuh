@@ -51,6 +51,8 @@ struct GemmParams {
     int32_t num_m_tiles;
     int32_t num_n_tiles;
     int32_t m_fastest;  // tile order: 1 = consecutive tiles share n (B panel)
+    int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
+    int32_t l2_b;
     int32_t *status;
 };
 
@@ -199,8 +201,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_b = policy_evict_last();
+            const uint64_t pol_a = policy_of(p.l2_a);
+            const uint64_t pol_b = policy_of(p.l2_b);
             uint32_t stage = 0, phase = 0;
             int64_t issued = 0;
             bool ok = true;

@@ -281,6 +281,8 @@ lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(K);
     p.m_fastest = 0;  // consecutive tiles share one W panel
+    p.l2_a = 1;       // W is streamed once (its panel's users run together)
+    p.l2_b = 2;       // X is reread by every tile
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, a, b, p, s)
@@ -308,6 +310,8 @@ lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(V);
     p.m_fastest = 1;
+    p.l2_a = 0;  // every W and dlogits chunk is read by the concurrently running tiles
+    p.l2_b = 0;
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<true, false, float>(bn, a, b, p, s)
@@ -335,6 +339,8 @@ lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t
     p.Ndim = static_cast<int32_t>(V);
     p.Kdim = static_cast<int32_t>(M);
     p.m_fastest = 1;  // consecutive tiles share one dlogits panel
+    p.l2_a = 2;       // X is reread by every tile
+    p.l2_b = 0;
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<true, true, float>(bn, a, b, p, s)

@@ -200,11 +200,24 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
+__device__ __forceinline__ uint64_t policy_evict_normal()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last()
 {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+
+// L2 policy by code: 0 normal, 1 evict first (streamed once), 2 evict last (reused).
+__device__ __forceinline__ uint64_t policy_of(int code)
+{
+    return code == 1 ? policy_evict_first() : code == 2 ? policy_evict_last() : policy_evict_normal();
 }
 
 // ---------------------------------------------------------------- tcgen05
