@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the workload the CPU oracle baseline processes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--step", choices=["separate", "fused"], default="separate",
+                    help="separate: the five calls; fused: lmhead_fwd_ce (logits and CE "
+                         "statistics in one pass) then ce_bwd, dX, dW")
     ap.add_argument("--workload", default="lmhead_1024x4096x32768",
                     choices=["lmhead_1024x4096x32768", "lmhead_4096x4096x128256",
                              "ce_8192x151936_outliers", "sweep"])
@@ -281,14 +284,25 @@ def run_ours(args, cfg):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    names = ["lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw"]
-    calls = [
-        lambda: lmhead.lmhead_fwd(Xd, Wd, logits, status),
-        lambda: lmhead.ce_fwd(logits, td, stats, -100, status),
-        lambda: lmhead.ce_bwd(logits, td, stats, gd, dl, -100, status),
-        lambda: lmhead.lmhead_bwd_dx(dl, Wd, dX, status),
-        lambda: lmhead.lmhead_bwd_dw(dl, Xd, dW, status),
-    ]
+    fused = args.step == "fused"
+    ws = torch.empty(lmhead.lmhead_fwd_ce_workspace_bytes(M, V), dtype=torch.uint8, device=dev)
+    if fused:
+        names = ["lmhead_fwd_ce", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw"]
+        calls = [
+            lambda: lmhead.lmhead_fwd_ce(Xd, Wd, td, logits, stats, ws, -100, status),
+            lambda: lmhead.ce_bwd(logits, td, stats, gd, dl, -100, status),
+            lambda: lmhead.lmhead_bwd_dx(dl, Wd, dX, status),
+            lambda: lmhead.lmhead_bwd_dw(dl, Xd, dW, status),
+        ]
+    else:
+        names = ["lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw"]
+        calls = [
+            lambda: lmhead.lmhead_fwd(Xd, Wd, logits, status),
+            lambda: lmhead.ce_fwd(logits, td, stats, -100, status),
+            lambda: lmhead.ce_bwd(logits, td, stats, gd, dl, -100, status),
+            lambda: lmhead.lmhead_bwd_dx(dl, Wd, dX, status),
+            lambda: lmhead.lmhead_bwd_dw(dl, Xd, dW, status),
+        ]
 
     def step():
         for c in calls:
@@ -345,8 +359,11 @@ def run_ours(args, cfg):
             tb[b].copy_(th, non_blocking=True)
             copied[b].record(cs)
         stream.wait_event(copied[b])
-        lmhead.lmhead_fwd(Xb[b], Wd, logits, status)
-        lmhead.ce_fwd(logits, tb[b], stats, -100, status)
+        if fused:
+            lmhead.lmhead_fwd_ce(Xb[b], Wd, tb[b], logits, stats, ws, -100, status)
+        else:
+            lmhead.lmhead_fwd(Xb[b], Wd, logits, status)
+            lmhead.ce_fwd(logits, tb[b], stats, -100, status)
         lmhead.ce_bwd(logits, tb[b], stats, gd, dl, -100, status)
         lmhead.lmhead_bwd_dx(dl, Wd, dX, status)
         lmhead.lmhead_bwd_dw(dl, Xb[b], dW, status)
@@ -375,7 +392,8 @@ def run_ours(args, cfg):
     nv = int((t != -100).sum())
     ce_fwd_bytes = nv * V * 4 + M * (8 + 16)
     ce_bwd_bytes = nv * V * 4 + M * V * 2 + M * (8 + 16)
-    algo = {"lmhead_fwd": ("tensor", flop), "ce_fwd": ("hbm", ce_fwd_bytes),
+    algo = {"lmhead_fwd": ("tensor", flop), "lmhead_fwd_ce": ("tensor", flop),
+            "ce_fwd": ("hbm", ce_fwd_bytes),
             "ce_bwd": ("hbm", ce_bwd_bytes), "lmhead_bwd_dx": ("tensor", flop),
             "lmhead_bwd_dw": ("tensor", flop)}
     traffic = committed_traffic()
@@ -404,13 +422,16 @@ def run_ours(args, cfg):
                        "dlogits": "bf16", "dX_dW": "fp32", "accumulate": "fp32",
                        "ignored_rows": M - nv, "grad_loss": "1/num_valid",
                        "l2": "flushed between steps (512 MiB write outside the timed events)",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}",
+                       "step": ("lmhead_fwd_ce, ce_bwd, lmhead_bwd_dx, lmhead_bwd_dw" if fused else
+                                "lmhead_fwd, ce_fwd, ce_bwd, lmhead_bwd_dx, lmhead_bwd_dw")},
             "roofline": roofline, "kernels": kernels,
             "e2e": {"value": world * M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "note": "pinned-host inputs copied on a second stream, double-buffered; "
                             "no L2 flush (the step's working set is far larger than L2)"},
-            "gpu_launches": len(calls) * K_steps, "clocks": clocks}
+            "gpu_launches": sum(2 if n == "lmhead_fwd_ce" else 1 for n in names) * K_steps,
+            "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of oracle work: the sample shrinks as the vocabulary grows
         sample = max(8, int(args.cpu_sample * 32768 * 4096 / (cfg.V * cfg.K)))

@@ -119,6 +119,31 @@ LMH_API lmh_status_t ce_bwd(const float *logits, const int64_t *target, const fl
                     int32_t dl_dtype, int64_t M, int64_t V, int64_t ignore_index,
                     int32_t *status, lmh_stream_t stream);
 
+/* logits = X . W^T (FP32) and the cross-entropy forward statistics of those
+ * logits in one pass over them: the vocabulary GEMM's epilogue reduces every
+ * 32-wide vocabulary slice of each token row to a partial (max, sum-exp) in
+ * `workspace` and records the target logit while the tile is still on chip,
+ * and a second kernel merges each token's partials (in a fixed order) into
+ * stats[M,4] = {m, d, x_y, loss}.  The logits are written but not read back
+ * -- the "one fewer read of the logits" of [P2] "Changes", taken one step
+ * further than a separate ce_fwd.
+ *   Arguments and results as lmhead_fwd (out_dtype FP32) followed by ce_fwd
+ *   (same tolerances; the statistics are merged in a different order, so they
+ *   need not be bitwise equal to ce_fwd's).
+ *   workspace: device scratch of at least lmhead_fwd_ce_workspace_bytes(M, V)
+ *   bytes, 16-byte aligned, owned by the caller; its contents on entry do not
+ *   matter and on return are unspecified.  When V % 4 != 0 or logits is not
+ *   16-byte aligned the call runs lmhead_fwd then ce_fwd and does not touch
+ *   the workspace (which may then be NULL). */
+LMH_API lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target,
+                                   float *logits, float *stats, void *workspace,
+                                   int64_t workspace_bytes, int64_t M, int64_t K, int64_t V,
+                                   int64_t ignore_index, int32_t *status, lmh_stream_t stream);
+
+/* Scratch bytes lmhead_fwd_ce needs: M tokens x 8 * ceil(V / 256) slices x
+ * 8 bytes (8 MB for M = 1024, V = 32768).  -1 for sizes out of range. */
+LMH_API int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V);
+
 /* dX = dlogits . W, the input gradient of logits = X . W^T
  * ([P1] "What does this PR do?", backward under the GEMM contract).
  *   dlogits [M,V] BF16.  W [V,K] BF16.
@@ -143,6 +168,15 @@ LMH_API const char *lmh_status_string(lmh_status_t s);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 LMH_API int32_t lmh_version(void);
+
+/* Self-test of the pipeline watchdog (failure detection; no counterpart on
+ * the pages).  Launches one CTA whose thread waits, with the same bounded
+ * wait the GEMM pipelines use, on a shared-memory barrier that nothing
+ * arrives at, with a limit of `limit_us` microseconds (1..1000000).  The wait
+ * gives up, the CTA unwinds and LMH_DEV_PIPE_TIMEOUT is ORed into *status
+ * (device int32, required).  Nothing faults or hangs; the context stays
+ * usable.  Asynchronous like every other call. */
+LMH_API lmh_status_t lmh_watchdog_selftest(int32_t *status, int64_t limit_us, lmh_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -14,31 +14,9 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "softmax_merge.cuh"
+
 namespace lmh {
-
-constexpr float kLog2e = 1.4426950408889634f;  // 1 / ln 2
-
-struct MaxSum {
-    float m;  // running maximum
-    float d;  // sum of exp(x - m)
-};
-
-// exp(t) for t <= 0, via the hardware base-2 exponential.
-__device__ __forceinline__ float exp_neg(float t) { return exp2f(t * kLog2e); }
-
-// Merge two (max, sum-exp) pairs: the associative step of the online softmax.
-__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b)
-{
-    if (a.m < b.m) {
-        MaxSum t = a;
-        a = b;
-        b = t;
-    }
-    // a.m >= b.m; b.m == -inf means b holds nothing
-    if (b.m == -INFINITY)
-        return a;
-    return MaxSum{a.m, a.d + b.d * exp_neg(b.m - a.m)};
-}
 
 // Fold a batch of N values into the running pair: one rescale per batch,
 // and the batch's own exponentials are summed first (short partial sums).
@@ -279,6 +257,56 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
                 const float v = load1<ALIAS>(x + j);
                 store1(o + j, (exp_neg(v - m) * inv_d - (j == y)) * g);
             }
+        }
+    }
+}
+
+// stats[i] = {m, d, x_y, loss} from the per-slice partials the fused
+// vocabulary GEMM wrote (partial[i * nslices + s]; the target logit is already
+// in stats[i].x_y).  One warp per token: lane l merges slices l, l + 32, ...
+// (eight 8-byte loads in flight), then the lanes are merged by a fixed
+// butterfly, so the result does not depend on scheduling.
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32)
+    ce_finalize_kernel(const float2 *__restrict__ partial, int64_t nslices,
+                       const int64_t *__restrict__ target, float4 *stats, int64_t M, int64_t V,
+                       int64_t ignore_index, int32_t *status)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t tok = static_cast<int64_t>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
+    if (tok >= M)
+        return;  // whole warp
+    const float2 *row = partial + tok * nslices;
+    MaxSum s{-INFINITY, 0.f};
+    int64_t sl = lane;
+    for (; sl + 7 * 32 < nslices; sl += 8 * 32) {
+        float2 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            v[u] = row[sl + u * 32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            s = merge(s, MaxSum{v[u].x, v[u].y});
+    }
+    for (; sl < nslices; sl += 32) {
+        const float2 v = row[sl];
+        s = merge(s, MaxSum{v.x, v.y});
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        MaxSum t{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.d, o)};
+        s = merge(s, t);
+    }
+    if (lane == 0) {
+        const int64_t y = target[tok];
+        const int kind = row_kind(y, V, ignore_index);
+        if (kind != 0) {
+            stats[tok] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kind == 2 && status)
+                atomicOr(status, 1);
+        } else {
+            const float xy = reinterpret_cast<const float *>(stats)[tok * 4 + 2];
+            stats[tok] = make_float4(s.m, s.d, xy, (s.m - xy) + logf(s.d));
         }
     }
 }

@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "softmax_merge.cuh"
 
 namespace lmh {
 
@@ -54,6 +55,13 @@ struct GemmParams {
     int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
     int32_t l2_b;
     int32_t *status;
+    // fused cross-entropy statistics (vocabulary GEMM only): per token i and
+    // 32-wide vocabulary slice s, ce_partial[i * ce_nslices + s] = (max,
+    // sum-exp) of the slice; the target logit goes to ce_stats[4 i + 2].
+    float2 *ce_partial;
+    int64_t ce_nslices;
+    const int64_t *ce_target;
+    float *ce_stats;
 };
 
 constexpr int kEpiWarps = 4;
@@ -130,6 +138,43 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt,
     }
 }
 
+// Partial cross-entropy statistics of one staged sub-tile (FP32 logits):
+// lane l takes token row l of the 32 x 32 box in shared memory (32 vocabulary
+// columns starting at vbase; columns at or past V excluded), reduces it to
+// (max, sum of exp(x - max)) and stores it for slice `slice`; the lane whose
+// row holds its token's target column also records the target logit.  The
+// columns are visited in a lane-rotated order, so the 32 lanes read 32
+// different banks.
+__device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int rows, int vbase,
+                                                 int V, int tok, int ntok, int64_t slice,
+                                                 const GemmParams &p)
+{
+    if (lane >= rows || tok >= ntok)
+        return;
+    const float *rowp = buf + lane * 32;
+    const int nvalid = V - vbase;  // may be <= 0 (a slice past the vocabulary) or > 32
+    float vmax = -INFINITY;
+#pragma unroll
+    for (int kk = 0; kk < 32; ++kk) {
+        const int col = (kk + lane) & 31;
+        if (col < nvalid)
+            vmax = fmaxf(vmax, rowp[col]);
+    }
+    float dsum = 0.f;
+    if (vmax != -INFINITY) {
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) {
+            const int col = (kk + lane) & 31;
+            if (col < nvalid)
+                dsum += exp_neg(rowp[col] - vmax);
+        }
+    }
+    p.ce_partial[static_cast<int64_t>(tok) * p.ce_nslices + slice] = make_float2(vmax, dsum);
+    const int64_t y = p.ce_target[tok];
+    if (y >= vbase && y < vbase + 32 && y < V)
+        p.ce_stats[static_cast<int64_t>(tok) * 4 + 2] = rowp[y - vbase];
+}
+
 // TMA_STORE: the output is written through tmC, a tensor map over
 // out[Ndim][ldo] with box {32, EPI_CHUNK}; otherwise by direct global stores.
 // PAIR: a cluster of two CTAs on one tile of 256 (m) x BN (n) with
@@ -137,7 +182,10 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt,
 // rows of B, the leader (rank 0) issues the MMAs, and each CTA's tensor
 // memory receives its 128 rows of the accumulator.  B is read from L2 once
 // per pair instead of once per SM.
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR>
+// CE (vocabulary GEMM, FP32 output, TMA_STORE): also emit the partial
+// cross-entropy statistics of every 32-wide vocabulary slice (see
+// ce_subtile_stats), so that the logits need not be read back.
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p)
@@ -381,6 +429,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (lane == 0) {
                         tma_store_2d(&tmC, buf, mbase + q * 32, n0 + c);
                         bulk_commit();
+                    }
+                    if constexpr (CE) {
+                        // the TMA store only reads the slot, so it can be read here too
+                        const int64_t slice =
+                            static_cast<int64_t>(mt * C::CTAS + static_cast<int>(rank)) * 4 + q;
+                        ce_subtile_stats(reinterpret_cast<const float *>(buf), lane, C::EPI_CHUNK,
+                                         mbase + q * 32, p.Mdim, n0 + c + lane, p.Ndim, slice, p);
                     }
                     slot ^= 1;
                 } else if (m_ok) {

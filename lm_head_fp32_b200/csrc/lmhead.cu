@@ -124,12 +124,12 @@ bool make_operand_map(CUtensorMap *map, const Operand &op, uint32_t rows)
 }
 
 // One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR>
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false>
 lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                               GemmParams p, cudaStream_t stream)
 {
     using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
-    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -216,6 +216,43 @@ bool use_pair(int bn, int64_t Mdim)
     return o < 0 ? true : o == 1;
 }
 
+// Vocabulary GEMM with the fused cross-entropy statistics (FP32 logits through
+// the TMA-store epilogue; the caller has checked that a tensor map can describe
+// them).  *nslices receives the number of 32-wide slices written.
+template <int BN, bool PAIR>
+lmh_status_t launch_gemm_ce(const Operand &a, const Operand &b, GemmParams p, int64_t *nslices,
+                            cudaStream_t stream)
+{
+    using C = GemmCfg<BN, false, false, PAIR>;
+    CUtensorMap ta, tb, tc;
+    if (!make_operand_map(&ta, a, lmh::kBlockM) || !make_operand_map(&tb, b, C::BN_CTA) ||
+        !make_out_map(&tc, p.out, false, static_cast<uint64_t>(p.Mdim),
+                      static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
+        return LMH_ERR_CUDA;
+    *nslices = 4 * static_cast<int64_t>(C::CTAS) * ((p.Mdim + C::TILE_M - 1) / C::TILE_M);
+    p.ce_nslices = *nslices;
+    return launch_gemm_impl<BN, false, false, float, true, PAIR, true>(ta, tb, tc, p, stream);
+}
+
+lmh_status_t dispatch_ce(int bn, const Operand &a, const Operand &b, GemmParams p, int64_t *nslices,
+                         cudaStream_t s)
+{
+    switch (bn) {
+    case 16: return launch_gemm_ce<16, false>(a, b, p, nslices, s);
+    case 32: return launch_gemm_ce<32, false>(a, b, p, nslices, s);
+    case 64: return launch_gemm_ce<64, false>(a, b, p, nslices, s);
+    case 128: return launch_gemm_ce<128, false>(a, b, p, nslices, s);
+    case 256:
+        return use_pair(bn, p.Mdim) ? launch_gemm_ce<256, true>(a, b, p, nslices, s)
+                                    : launch_gemm_ce<256, false>(a, b, p, nslices, s);
+    default: return LMH_ERR_UNSUPPORTED;
+    }
+}
+
+// Slices of partial statistics the fused GEMM may write for a vocabulary of V
+// (both tile modes fit: 8 per 256 vocabulary columns).
+int64_t ce_slices(int64_t V) { return 8 * ((V + 255) / 256); }
+
 template <bool A_MN, bool B_MN, typename OutT>
 lmh_status_t dispatch_bn(int bn, const Operand &a, const Operand &b, GemmParams p, cudaStream_t s)
 {
@@ -237,6 +274,23 @@ lmh_status_t dispatch_bn(int bn, const Operand &a, const Operand &b, GemmParams 
 }
 
 bool bad_dtype(int32_t t) { return t != LMH_F32 && t != LMH_BF16; }
+
+// One thread waits on a barrier that expects an arrival nobody makes.
+__global__ void watchdog_selftest_kernel(int32_t *status, uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        lmh::mbar_init(&bar, 1);
+        abort_flag = 0;
+        lmh::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (!lmh::mbar_wait(&bar, 0, &abort_flag, limit_ns))
+            atomicOr(status, LMH_DEV_PIPE_TIMEOUT);
+    }
+}
 
 bool dims_ok(int64_t a, int64_t b, int64_t c)
 {
@@ -260,6 +314,15 @@ const char *lmh_status_string(lmh_status_t s)
 }
 
 int32_t lmh_version(void) { return 100; }
+
+lmh_status_t lmh_watchdog_selftest(int32_t *status, int64_t limit_us, lmh_stream_t stream)
+{
+    if (!status || limit_us < 1 || limit_us > 1000000)
+        return LMH_ERR_INVALID_ARG;
+    watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        status, static_cast<uint64_t>(limit_us) * 1000ull);
+    return last_cuda_error();
+}
 
 lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_dtype, int64_t M,
                         int64_t K, int64_t V, int32_t *status, lmh_stream_t stream)
@@ -345,6 +408,61 @@ lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<true, true, float>(bn, a, b, p, s)
                                 : dispatch_bn<true, true, __nv_bfloat16>(bn, a, b, p, s);
+}
+
+int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V)
+{
+    if (M < 1 || V < 1 || M > kMaxDim || V > kMaxDim)
+        return -1;
+    return ce_slices(V) * M * static_cast<int64_t>(sizeof(float2));
+}
+
+lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target, float *logits,
+                           float *stats, void *workspace, int64_t workspace_bytes, int64_t M,
+                           int64_t K, int64_t V, int64_t ignore_index, int32_t *status,
+                           lmh_stream_t stream)
+{
+    if (!X || !W || !target || !logits || !stats || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (K % 8 || !aligned(X, 16) || !aligned(W, 16) || !aligned(logits, 4) || !aligned(target, 8) ||
+        !aligned(stats, 16))
+        return LMH_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (V % 4 != 0 || !aligned(logits, 16)) {
+        // logits a tensor map cannot describe: the two separate passes
+        const lmh_status_t r = lmhead_fwd(X, W, logits, LMH_F32, M, K, V, status, stream);
+        return r != LMH_OK ? r : ce_fwd(logits, target, stats, M, V, ignore_index, status, stream);
+    }
+    if (!workspace || workspace_bytes < lmhead_fwd_ce_workspace_bytes(M, V))
+        return LMH_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16))
+        return LMH_ERR_MISALIGNED;
+    const int bn = pick_bn_tokens(M);
+    const Operand a{W, static_cast<uint64_t>(K), static_cast<uint64_t>(V), false};
+    const Operand b{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), false};
+    GemmParams p{};
+    p.out = logits;
+    p.ldo = V;
+    p.Mdim = static_cast<int32_t>(V);
+    p.Ndim = static_cast<int32_t>(M);
+    p.Kdim = static_cast<int32_t>(K);
+    p.m_fastest = 0;
+    p.l2_a = 1;
+    p.l2_b = 2;
+    p.status = status;
+    p.ce_partial = static_cast<float2 *>(workspace);
+    p.ce_target = target;
+    p.ce_stats = stats;
+    int64_t nslices = 0;
+    const lmh_status_t r = dispatch_ce(bn, a, b, p, &nslices, s);
+    if (r != LMH_OK)
+        return r;
+    constexpr int kFinalizeWarps = 8;  // tokens per CTA
+    const int64_t grid = (M + kFinalizeWarps - 1) / kFinalizeWarps;
+    lmh::ce_finalize_kernel<kFinalizeWarps><<<static_cast<unsigned>(grid), kFinalizeWarps * 32, 0, s>>>(
+        static_cast<const float2 *>(workspace), nslices, target, reinterpret_cast<float4 *>(stats), M,
+        V, ignore_index, status);
+    return last_cuda_error();
 }
 
 lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, int64_t M, int64_t V,

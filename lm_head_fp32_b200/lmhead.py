@@ -23,7 +23,8 @@ DEV_PIPE_TIMEOUT = 0x2
 IGNORE_INDEX = -100
 
 EXPORTS = ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
-           "lmh_status_string", "lmh_version")
+           "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes",
+           "lmh_status_string", "lmh_version", "lmh_watchdog_selftest")
 
 _lib = None
 
@@ -53,6 +54,12 @@ def lib() -> ctypes.CDLL:
         L.lmh_status_string.argtypes = [ctypes.c_int]
         L.lmh_status_string.restype = ctypes.c_char_p
         L.lmh_version.restype = ctypes.c_int32
+        L.lmhead_fwd_ce.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P]
+        L.lmhead_fwd_ce.restype = ctypes.c_int
+        L.lmhead_fwd_ce_workspace_bytes.argtypes = [I64, I64]
+        L.lmhead_fwd_ce_workspace_bytes.restype = I64
+        L.lmh_watchdog_selftest.argtypes = [P, I64, P]
+        L.lmh_watchdog_selftest.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -132,6 +139,30 @@ def ce_bwd(logits: torch.Tensor, target: torch.Tensor, stats: torch.Tensor,
     return dlogits
 
 
+def lmhead_fwd_ce_workspace_bytes(M: int, V: int) -> int:
+    """Scratch bytes lmhead_fwd_ce needs for M tokens and a vocabulary of V."""
+    return int(lib().lmhead_fwd_ce_workspace_bytes(int(M), int(V)))
+
+
+def lmhead_fwd_ce(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor, logits: torch.Tensor,
+                  stats: torch.Tensor, workspace: torch.Tensor,
+                  ignore_index: int = IGNORE_INDEX, status: Optional[torch.Tensor] = None,
+                  stream=None):
+    """FP32 logits = X . W^T and stats[M,4] = {m, d, x_y, loss} in one pass over
+    the logits; `workspace` is caller-owned scratch (uint8, see
+    lmhead_fwd_ce_workspace_bytes)."""
+    _contig(X, W, target, logits, stats, workspace)
+    M, K = X.shape
+    V = W.shape[0]
+    assert W.shape[1] == K and tuple(logits.shape) == (M, V) and tuple(stats.shape) == (M, 4)
+    assert logits.dtype == torch.float32
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().lmhead_fwd_ce(_ptr(X), _ptr(W), _ptr(target), _ptr(logits), _ptr(stats),
+                               _ptr(workspace), nbytes, M, K, V, int(ignore_index), _ptr(status),
+                               _stream(stream)), "lmhead_fwd_ce")
+    return logits, stats
+
+
 def lmhead_bwd_dx(dlogits: torch.Tensor, W: torch.Tensor, dX: torch.Tensor,
                   status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """dX[M,K] = dlogits[M,V] . W[V,K]."""
@@ -154,3 +185,9 @@ def lmhead_bwd_dw(dlogits: torch.Tensor, X: torch.Tensor, dW: torch.Tensor,
     _check(lib().lmhead_bwd_dw(_ptr(dlogits), _ptr(X), _ptr(dW), _dtype_code(dW.dtype),
                                M, K, V, _ptr(status), _stream(stream)), "lmhead_bwd_dw")
     return dW
+
+
+def watchdog_selftest(status: torch.Tensor, limit_us: int = 1000, stream=None) -> None:
+    """Make one bounded pipeline wait run out on purpose; sets DEV_PIPE_TIMEOUT."""
+    _check(lib().lmh_watchdog_selftest(_ptr(status), int(limit_us), _stream(stream)),
+           "lmh_watchdog_selftest")

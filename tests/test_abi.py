@@ -28,7 +28,7 @@ def declared_functions():
 def test_header_declares_the_five_calls():
     fns = declared_functions()
     for f in ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
-              "lmh_status_string"):
+              "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes", "lmh_status_string"):
         assert f in fns
 
 
@@ -100,3 +100,29 @@ def test_binding_rejects_fp16_like_the_flag():
     assert lmhead._dtype_code(torch.float16) == lmhead.F16
     with pytest.raises(TypeError):
         lmhead._dtype_code(torch.int8)
+
+
+def test_watchdog_selftest_validation():
+    L = lmhead.lib()
+    assert L.lmh_watchdog_selftest(NULL, 1000, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert L.lmh_watchdog_selftest(A, 0, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert L.lmh_watchdog_selftest(A, 2000000, NULL) == lmhead.LMH_ERR_INVALID_ARG
+
+
+def test_fused_ce_workspace_size_and_validation():
+    L = lmhead.lib()
+    assert lmhead.lmhead_fwd_ce_workspace_bytes(1024, 32768) == 8 * 128 * 1024 * 8
+    assert lmhead.lmhead_fwd_ce_workspace_bytes(16, 1) == 8 * 1 * 16 * 8
+    assert lmhead.lmhead_fwd_ce_workspace_bytes(0, 10) == -1
+    f = L.lmhead_fwd_ce
+    need = lmhead.lmhead_fwd_ce_workspace_bytes(16, 64)
+    assert f(NULL, A, A, A, A, A, need, 16, 64, 64, -100, NULL, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, A, need, 16, 60, 64, -100, NULL, NULL) == lmhead.LMH_ERR_MISALIGNED
+    assert f(A, A, A, A, P(0x10008), A, need, 16, 64, 64, -100, NULL, NULL) == \
+        lmhead.LMH_ERR_MISALIGNED                     # stats not 16-byte aligned
+    # the fused path needs the workspace (V % 4 == 0, aligned logits)
+    assert f(A, A, A, A, A, NULL, need, 16, 64, 64, -100, NULL, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, A, need - 8, 16, 64, 64, -100, NULL, NULL) == \
+        lmhead.LMH_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, P(0x10008), need, 16, 64, 64, -100, NULL, NULL) == \
+        lmhead.LMH_ERR_MISALIGNED
