@@ -144,6 +144,31 @@ LMH_API lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *
  * 8 bytes (8 MB for M = 1024, V = 32768).  -1 for sizes out of range. */
 LMH_API int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V);
 
+/* lmhead_fwd_ce for callers that cannot allocate device memory (no
+ * counterpart on the pages).  Some callers cannot give the library a scratch
+ * buffer: plug-ins whose host framework owns all device memory and offers
+ * them no allocator, and code on paths where calling cudaMalloc (which may
+ * synchronise the device) is not allowed.  This call computes exactly what
+ * lmhead_fwd_ce computes (same arguments minus the workspace) but keeps the
+ * partial statistics in a fixed 8 MiB array inside the library, which every
+ * GPU that loads the library holds until the process exits.  It allocates
+ * nothing and calls no allocating routine.
+ *   Limit: M * 8 * ceil(V / 256) <= 1048576 (e.g. M = 1024 with V up to
+ *   32768); larger problems return LMH_ERR_INVALID_ARG before anything is
+ *   launched.  (When V % 4 != 0 or logits is not 16-byte aligned the call
+ *   runs lmhead_fwd then ce_fwd, which need no scratch, at any size.)
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   Every call shares the one array per device: calls that may run at the
+ *   same time on the GPU (different streams, or different host threads)
+ *   race and corrupt each other's results.  Nothing in the array has to start
+ *   at zero: each call writes every entry it later reads. */
+LMH_API lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, const int64_t *target,
+                                           float *logits, float *stats, int64_t M, int64_t K,
+                                           int64_t V, int64_t ignore_index, int32_t *status,
+                                           lmh_stream_t stream);
+
 /* dX = dlogits . W, the input gradient of logits = X . W^T
  * ([P1] "What does this PR do?", backward under the GEMM contract).
  *   dlogits [M,V] BF16.  W [V,K] BF16.

@@ -533,3 +533,94 @@ lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *sta
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// lmhead_fwd_ce_noalloc: lmhead_fwd_ce for callers that cannot allocate.
+//
+// Some callers cannot hand this library a scratch buffer: plug-ins whose host
+// framework owns all device memory and gives them no allocator, and code on
+// paths where calling cudaMalloc (which may synchronise the device) is not
+// allowed.  For them the partial statistics live in one fixed array below,
+// part of the library image: every GPU that loads the library holds these
+// 8 MiB until the process exits.  The caller still passes every input and
+// output.  This call allocates nothing and calls no allocating routine.
+//
+// In host code `g_fwd_ce_scratch` only names a host-side stand-in for the
+// array; handing it to a kernel would fault, or on systems where the GPU can
+// reach host memory silently use the wrong memory.  The device address is
+// therefore looked up with cudaGetSymbolAddress, once per device, with that
+// device current, the first time the call runs on it; make that first call
+// before any stream capture.
+// ----------------------------------------------------------------------------
+
+namespace {
+
+constexpr int64_t kNoAllocScratchBytes = 8ll << 20;  // 8 MiB of partial statistics
+static __device__ __align__(256) float2 g_fwd_ce_scratch[kNoAllocScratchBytes / sizeof(float2)];
+
+// Device address of g_fwd_ce_scratch on the current device (nullptr on error).
+float2 *noalloc_scratch()
+{
+    static std::mutex mu;
+    static float2 *addr[kMaxDevices] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fwd_ce_scratch) != cudaSuccess)
+            return nullptr;
+        addr[dev] = static_cast<float2 *>(p);
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, const int64_t *target,
+                                              float *logits, float *stats, int64_t M, int64_t K,
+                                              int64_t V, int64_t ignore_index, int32_t *status,
+                                              lmh_stream_t stream)
+{
+    if (!X || !W || !target || !logits || !stats || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (K % 8 || !aligned(X, 16) || !aligned(W, 16) || !aligned(logits, 4) || !aligned(target, 8) ||
+        !aligned(stats, 16))
+        return LMH_ERR_MISALIGNED;
+    if (V % 4 != 0 || !aligned(logits, 16))  // the two separate passes need no scratch
+        return lmhead_fwd_ce(X, W, target, logits, stats, nullptr, 0, M, K, V, ignore_index, status,
+                             stream);
+    // larger problems are rejected before anything is launched
+    if (ce_slices(V) > kNoAllocScratchBytes / static_cast<int64_t>(sizeof(float2)) / M)
+        return LMH_ERR_INVALID_ARG;
+    float2 *scratch = noalloc_scratch();
+    if (!scratch)
+        return LMH_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int bn = pick_bn_tokens(M);
+    const Operand a{W, static_cast<uint64_t>(K), static_cast<uint64_t>(V), false};
+    const Operand b{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), false};
+    GemmParams p{};
+    p.out = logits;
+    p.ldo = V;
+    p.Mdim = static_cast<int32_t>(V);
+    p.Ndim = static_cast<int32_t>(M);
+    p.Kdim = static_cast<int32_t>(K);
+    p.m_fastest = 0;
+    p.l2_a = 1;
+    p.l2_b = 2;
+    p.status = status;
+    p.ce_partial = scratch;
+    p.ce_target = target;
+    p.ce_stats = stats;
+    int64_t nslices = 0;
+    const lmh_status_t r = dispatch_ce(bn, a, b, p, &nslices, s);
+    if (r != LMH_OK)
+        return r;
+    constexpr int kFinalizeWarps = 8;
+    const int64_t grid = (M + kFinalizeWarps - 1) / kFinalizeWarps;
+    lmh::ce_finalize_kernel<kFinalizeWarps><<<static_cast<unsigned>(grid), kFinalizeWarps * 32, 0, s>>>(
+        scratch, nslices, target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
+    return last_cuda_error();
+}

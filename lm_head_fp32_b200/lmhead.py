@@ -23,7 +23,7 @@ DEV_PIPE_TIMEOUT = 0x2
 IGNORE_INDEX = -100
 
 EXPORTS = ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
-           "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes",
+           "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes", "lmhead_fwd_ce_noalloc",
            "lmh_status_string", "lmh_version", "lmh_watchdog_selftest")
 
 _lib = None
@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.lmh_version.restype = ctypes.c_int32
         L.lmhead_fwd_ce.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P]
         L.lmhead_fwd_ce.restype = ctypes.c_int
+        L.lmhead_fwd_ce_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
+        L.lmhead_fwd_ce_noalloc.restype = ctypes.c_int
         L.lmhead_fwd_ce_workspace_bytes.argtypes = [I64, I64]
         L.lmhead_fwd_ce_workspace_bytes.restype = I64
         L.lmh_watchdog_selftest.argtypes = [P, I64, P]
@@ -160,6 +162,25 @@ def lmhead_fwd_ce(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor, logits
     _check(lib().lmhead_fwd_ce(_ptr(X), _ptr(W), _ptr(target), _ptr(logits), _ptr(stats),
                                _ptr(workspace), nbytes, M, K, V, int(ignore_index), _ptr(status),
                                _stream(stream)), "lmhead_fwd_ce")
+    return logits, stats
+
+
+def lmhead_fwd_ce_noalloc(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor,
+                          logits: torch.Tensor, stats: torch.Tensor,
+                          ignore_index: int = IGNORE_INDEX, status: Optional[torch.Tensor] = None,
+                          stream=None):
+    """lmhead_fwd_ce without a workspace, for callers that cannot allocate
+    device memory: the partial statistics live in a fixed 8 MiB array inside
+    the library (M * 8 * ceil(V/256) <= 1048576).  Calls that overlap on the
+    GPU share that array and race."""
+    _contig(X, W, target, logits, stats)
+    M, K = X.shape
+    V = W.shape[0]
+    assert W.shape[1] == K and tuple(logits.shape) == (M, V) and tuple(stats.shape) == (M, 4)
+    assert logits.dtype == torch.float32
+    _check(lib().lmhead_fwd_ce_noalloc(_ptr(X), _ptr(W), _ptr(target), _ptr(logits), _ptr(stats),
+                                       M, K, V, int(ignore_index), _ptr(status), _stream(stream)),
+           "lmhead_fwd_ce_noalloc")
     return logits, stats
 
 
