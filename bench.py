@@ -315,7 +315,10 @@ def run_ours(args, cfg):
     assert int(status.item()) == 0, f"device status {int(status.item())}"
 
     K_steps = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K_steps)]
+    # one event before each step and one after every call: the step time and
+    # the per-kernel times come from the same loop (the same clocks and power)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+          for _ in range(K_steps)]
     sampler = ClockSampler(dev.index)
     barrier(pg)
     torch.cuda.synchronize()
@@ -331,7 +334,8 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     barrier(pg)
-    per_call = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_steps)] for j in range(len(calls))]
+    per_call = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_steps)]
+                for j in range(len(calls))]
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(K_steps)]
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"

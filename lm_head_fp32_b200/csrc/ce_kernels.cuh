@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "ptx.cuh"
 #include "softmax_merge.cuh"
 
 namespace lmh {
@@ -120,6 +121,8 @@ __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict
                                                             int32_t *status)
 {
     __shared__ MaxSum red[32];
+    pdl_wait();  // the logits may come from the kernel just before this one
+    pdl_launch_dependents();
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
         const int64_t y = target[row];
         const int kind = row_kind(y, V, ignore_index);
@@ -201,6 +204,8 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
     const float *__restrict__ grad_loss, int64_t grad_stride, OutT *dl, int64_t M, int64_t V,
     int64_t ignore_index, int32_t *status)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     // rows in the opposite order to ce_fwd: the rows it read last are the
     // ones most likely still in L2
     for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
@@ -272,6 +277,8 @@ __global__ void __launch_bounds__(WARPS * 32)
                        const int64_t *__restrict__ target, float4 *stats, int64_t M, int64_t V,
                        int64_t ignore_index, int32_t *status)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t tok = static_cast<int64_t>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
     if (tok >= M)

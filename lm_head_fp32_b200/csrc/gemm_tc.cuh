@@ -245,6 +245,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // everything above overlaps the previous kernel's tail; inputs and
+    // outputs are touched only after it has completed
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer

@@ -106,6 +106,50 @@ lmh_status_t last_cuda_error()
     return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
 
+// Programmatic dependent launch is on unless LMH_PDL=0 is set in the
+// environment (a tuning aid; read once per process).
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char *e = std::getenv("LMH_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+// Launch with programmatic stream serialisation allowed (the kernel waits in
+// pdl_wait before touching memory the previous kernel may still write) and,
+// for cluster_x > 1, thread-block clusters of cluster_x CTAs.
+template <typename... KArgs, typename... Args>
+lmh_status_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, unsigned cluster_x, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess)
+        return LMH_ERR_CUDA;
+    return last_cuda_error();
+}
+
 // A GEMM operand as a 2-D BF16 tensor [outer][inner] (inner contiguous).
 // mn_major: the inner dimension is the operand's m (or n) dimension and the
 // outer one its reduction dimension; otherwise the reverse.
@@ -148,25 +192,8 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
         return LMH_ERR_INVALID_ARG;
     const int64_t units = num_sms() / C::CTAS;  // CTAs (or CTA pairs) resident at once
     const int grid = static_cast<int>((tiles < units ? tiles : units) * C::CTAS);
-    if (PAIR) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid, 1, 1);
-        cfg.blockDim = dim3(lmh::kGemmThreads, 1, 1);
-        cfg.dynamicSmemBytes = C::SMEM_BYTES;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p) != cudaSuccess)
-            return LMH_ERR_CUDA;
-    } else {
-        kern<<<grid, lmh::kGemmThreads, C::SMEM_BYTES, stream>>>(ta, tb, tc, p);
-    }
-    return last_cuda_error();
+    return launch_ex(kern, dim3(grid), dim3(lmh::kGemmThreads), C::SMEM_BYTES, stream,
+                     PAIR ? 2u : 1u, ta, tb, tc, p);
 }
 
 template <int BN, bool A_MN, bool B_MN, typename OutT, bool PAIR>
@@ -459,10 +486,9 @@ lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target, 
         return r;
     constexpr int kFinalizeWarps = 8;  // tokens per CTA
     const int64_t grid = (M + kFinalizeWarps - 1) / kFinalizeWarps;
-    lmh::ce_finalize_kernel<kFinalizeWarps><<<static_cast<unsigned>(grid), kFinalizeWarps * 32, 0, s>>>(
-        static_cast<const float2 *>(workspace), nslices, target, reinterpret_cast<float4 *>(stats), M,
-        V, ignore_index, status);
-    return last_cuda_error();
+    return launch_ex(lmh::ce_finalize_kernel<kFinalizeWarps>, dim3(static_cast<unsigned>(grid)),
+                     dim3(kFinalizeWarps * 32), 0, s, 1u, static_cast<const float2 *>(workspace),
+                     nslices, target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
 }
 
 lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, int64_t M, int64_t V,
@@ -478,10 +504,10 @@ lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, in
     const bool vec = (V % 4 == 0) && aligned(logits, 16);
     float4 *st4 = reinterpret_cast<float4 *>(stats);
     if (vec)
-        lmh::ce_fwd_kernel<true, kCeThreads><<<grid, kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
-    else
-        lmh::ce_fwd_kernel<false, kCeThreads><<<grid, kCeThreads, 0, s>>>(logits, target, st4, M, V, ignore_index, status);
-    return last_cuda_error();
+        return launch_ex(lmh::ce_fwd_kernel<true, kCeThreads>, dim3(grid), dim3(kCeThreads), 0, s, 1u,
+                         logits, target, st4, M, V, ignore_index, status);
+    return launch_ex(lmh::ce_fwd_kernel<false, kCeThreads>, dim3(grid), dim3(kCeThreads), 0, s, 1u,
+                     logits, target, st4, M, V, ignore_index, status);
 }
 
 lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *stats,
@@ -507,29 +533,19 @@ lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *sta
         float *o = static_cast<float *>(dlogits);
         const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 16);
         const bool alias = static_cast<const void *>(logits) == dlogits;
-        if (vec && alias)
-            lmh::ce_bwd_kernel<float, true, true, kCeThreads><<<grid, kCeThreads, 0, s>>>(
-                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
-        else if (vec)
-            lmh::ce_bwd_kernel<float, true, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
-                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
-        else if (alias)
-            lmh::ce_bwd_kernel<float, false, true, kCeThreads><<<grid, kCeThreads, 0, s>>>(
-                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
-        else
-            lmh::ce_bwd_kernel<float, false, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
-                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
-    } else {
-        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(dlogits);
-        const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 8);
-        if (vec)
-            lmh::ce_bwd_kernel<__nv_bfloat16, true, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
-                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
-        else
-            lmh::ce_bwd_kernel<__nv_bfloat16, false, false, kCeThreads><<<grid, kCeThreads, 0, s>>>(
-                logits, target, st4, grad_loss, grad_loss_stride, o, M, V, ignore_index, status);
+        auto k = vec ? (alias ? lmh::ce_bwd_kernel<float, true, true, kCeThreads>
+                              : lmh::ce_bwd_kernel<float, true, false, kCeThreads>)
+                     : (alias ? lmh::ce_bwd_kernel<float, false, true, kCeThreads>
+                              : lmh::ce_bwd_kernel<float, false, false, kCeThreads>);
+        return launch_ex(k, dim3(grid), dim3(kCeThreads), 0, s, 1u, logits, target, st4, grad_loss,
+                         grad_loss_stride, o, M, V, ignore_index, status);
     }
-    return last_cuda_error();
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(dlogits);
+    const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 8);
+    auto k = vec ? lmh::ce_bwd_kernel<__nv_bfloat16, true, false, kCeThreads>
+                 : lmh::ce_bwd_kernel<__nv_bfloat16, false, false, kCeThreads>;
+    return launch_ex(k, dim3(grid), dim3(kCeThreads), 0, s, 1u, logits, target, st4, grad_loss,
+                     grad_loss_stride, o, M, V, ignore_index, status);
 }
 
 }  // extern "C"
@@ -620,7 +636,7 @@ extern "C" lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, cons
         return r;
     constexpr int kFinalizeWarps = 8;
     const int64_t grid = (M + kFinalizeWarps - 1) / kFinalizeWarps;
-    lmh::ce_finalize_kernel<kFinalizeWarps><<<static_cast<unsigned>(grid), kFinalizeWarps * 32, 0, s>>>(
-        scratch, nslices, target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
-    return last_cuda_error();
+    return launch_ex(lmh::ce_finalize_kernel<kFinalizeWarps>, dim3(static_cast<unsigned>(grid)),
+                     dim3(kFinalizeWarps * 32), 0, s, 1u, static_cast<const float2 *>(scratch), nslices,
+                     target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
 }

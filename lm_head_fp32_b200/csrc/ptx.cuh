@@ -131,6 +131,19 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 
 __device__ __forceinline__ void sleep_ns(uint32_t ns) { asm volatile("nanosleep.u32 %0;" ::"r"(ns)); }
 
+// ------------------------------------------- programmatic dependent launch
+
+// Block until the grids this one depends on have completed and their memory
+// is visible (returns at once when the launch did not allow overlap).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid on the stream to begin launching (its CTAs still wait
+// in pdl_wait for this grid to complete).
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
