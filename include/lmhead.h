@@ -188,6 +188,18 @@ LMH_API lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW,
                            int64_t M, int64_t K, int64_t V, int32_t *status,
                            lmh_stream_t stream);
 
+/* dW += dlogits^T . X: the weight gradient accumulated into an FP32 main
+ * gradient (beta = 1), as when gradients of several micro-batches are summed
+ * before the optimizer step.
+ *   dlogits [M,V] BF16, X [M,K] BF16, dW [V,K] FP32 (read and written).
+ *   Each dW element receives exactly one FP32 addition per call (performed
+ *   by the TMA reduce-add of the epilogue, or one atomic add where a tensor
+ *   map cannot describe dW), so the result does not depend on scheduling:
+ *   dW_out = fl(dW_in + fl32-accumulated product).
+ *   Requirements as lmhead_bwd_dw. */
+LMH_API lmh_status_t lmhead_bwd_dw_acc(const void *dlogits, const void *X, float *dW, int64_t M,
+                                       int64_t K, int64_t V, int32_t *status, lmh_stream_t stream);
+
 /* Static, NUL-terminated description of a status value. */
 LMH_API const char *lmh_status_string(lmh_status_t s);
 

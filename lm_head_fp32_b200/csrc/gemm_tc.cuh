@@ -185,7 +185,10 @@ __device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int
 // CE (vocabulary GEMM, FP32 output, TMA_STORE): also emit the partial
 // cross-entropy statistics of every 32-wide vocabulary slice (see
 // ce_subtile_stats), so that the logits need not be read back.
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false>
+// ACC (FP32 output): add the product to the output instead of overwriting it
+// (TMA reduce-add, or one atomic add per element on the direct path).
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
+          bool ACC = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p)
@@ -431,7 +434,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmC, buf, mbase + q * 32, n0 + c);
+                        if (ACC)
+                            tma_reduce_add_2d(&tmC, buf, mbase + q * 32, n0 + c);
+                        else
+                            tma_store_2d(&tmC, buf, mbase + q * 32, n0 + c);
                         bulk_commit();
                     }
                     if constexpr (CE) {
@@ -446,8 +452,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     OutT *o = out + static_cast<int64_t>(n0 + c) * p.ldo + m;
 #pragma unroll
                     for (int j = 0; j < C::EPI_CHUNK; ++j)
-                        if (n0 + c + j < p.Ndim)
-                            store_out(o + static_cast<int64_t>(j) * p.ldo, r[j]);
+                        if (n0 + c + j < p.Ndim) {
+                            if constexpr (ACC)
+                                atomicAdd(reinterpret_cast<float *>(o) + static_cast<int64_t>(j) * p.ldo,
+                                          __uint_as_float(r[j]));
+                            else
+                                store_out(o + static_cast<int64_t>(j) * p.ldo, r[j]);
+                        }
                 }
             }
             tc_fence_before();

@@ -168,12 +168,13 @@ bool make_operand_map(CUtensorMap *map, const Operand &op, uint32_t rows)
 }
 
 // One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false>
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
+          bool ACC = false>
 lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                               GemmParams p, cudaStream_t stream)
 {
     using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
-    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE, ACC>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -208,6 +209,21 @@ lmh_status_t launch_gemm(const Operand &a, const Operand &b, GemmParams p, cudaS
         return launch_gemm_impl<BN, A_MN, B_MN, OutT, true, PAIR>(ta, tb, tc, p, stream);
     std::memset(&tc, 0, sizeof tc);
     return launch_gemm_impl<BN, A_MN, B_MN, OutT, false, PAIR>(ta, tb, tc, p, stream);
+}
+
+// dW += dlogits^T . X (FP32): the dW GEMM with an accumulating epilogue.
+template <int BN, bool PAIR>
+lmh_status_t launch_dw_acc(const Operand &a, const Operand &b, GemmParams p, cudaStream_t stream)
+{
+    using C = GemmCfg<BN, true, true, PAIR>;
+    CUtensorMap ta, tb, tc;
+    if (!make_operand_map(&ta, a, lmh::kBlockM) || !make_operand_map(&tb, b, C::BN_CTA))
+        return LMH_ERR_CUDA;
+    if (make_out_map(&tc, p.out, false, static_cast<uint64_t>(p.Mdim),
+                     static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
+        return launch_gemm_impl<BN, true, true, float, true, PAIR, false, true>(ta, tb, tc, p, stream);
+    std::memset(&tc, 0, sizeof tc);
+    return launch_gemm_impl<BN, true, true, float, false, PAIR, false, true>(ta, tb, tc, p, stream);
 }
 
 // Token-dimension tile width for the vocabulary GEMM and dX: the smallest
@@ -435,6 +451,36 @@ lmh_status_t lmhead_bwd_dw(const void *dlogits, const void *X, void *dW, int32_t
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<true, true, float>(bn, a, b, p, s)
                                 : dispatch_bn<true, true, __nv_bfloat16>(bn, a, b, p, s);
+}
+
+lmh_status_t lmhead_bwd_dw_acc(const void *dlogits, const void *X, float *dW, int64_t M, int64_t K,
+                               int64_t V, int32_t *status, lmh_stream_t stream)
+{
+    if (!dlogits || !X || !dW || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (K % 8 || V % 8 || !aligned(dlogits, 16) || !aligned(X, 16) || !aligned(dW, 4))
+        return LMH_ERR_MISALIGNED;
+    const int bn = V <= 64 ? 64 : V <= 128 ? 128 : 256;
+    const Operand a{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), true};
+    const Operand b{dlogits, static_cast<uint64_t>(V), static_cast<uint64_t>(M), true};
+    GemmParams p{};
+    p.out = dW;
+    p.ldo = K;
+    p.Mdim = static_cast<int32_t>(K);
+    p.Ndim = static_cast<int32_t>(V);
+    p.Kdim = static_cast<int32_t>(M);
+    p.m_fastest = 1;
+    p.l2_a = 2;
+    p.l2_b = 0;
+    p.status = status;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (bn) {
+    case 64: return launch_dw_acc<64, false>(a, b, p, s);
+    case 128: return launch_dw_acc<128, false>(a, b, p, s);
+    default:
+        return use_pair(bn, p.Mdim) ? launch_dw_acc<256, true>(a, b, p, s)
+                                    : launch_dw_acc<256, false>(a, b, p, s);
+    }
 }
 
 int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V)

@@ -187,6 +187,18 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
                  : "memory");
 }
 
+// As tma_store_2d, but each element of the box is added to global memory
+// (one atomic FP32 add per element, performed at L2).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, const void *src,
+                                                  int32_t c0, int32_t c1)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N bulk groups still read their shared-memory source.

@@ -24,6 +24,7 @@ IGNORE_INDEX = -100
 
 EXPORTS = ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
            "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes", "lmhead_fwd_ce_noalloc",
+           "lmhead_bwd_dw_acc",
            "lmh_status_string", "lmh_version", "lmh_watchdog_selftest")
 
 _lib = None
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.lmh_version.restype = ctypes.c_int32
         L.lmhead_fwd_ce.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P]
         L.lmhead_fwd_ce.restype = ctypes.c_int
+        L.lmhead_bwd_dw_acc.argtypes = [P, P, P, I64, I64, I64, P, P]
+        L.lmhead_bwd_dw_acc.restype = ctypes.c_int
         L.lmhead_fwd_ce_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
         L.lmhead_fwd_ce_noalloc.restype = ctypes.c_int
         L.lmhead_fwd_ce_workspace_bytes.argtypes = [I64, I64]
@@ -212,3 +215,15 @@ def watchdog_selftest(status: torch.Tensor, limit_us: int = 1000, stream=None) -
     """Make one bounded pipeline wait run out on purpose; sets DEV_PIPE_TIMEOUT."""
     _check(lib().lmh_watchdog_selftest(_ptr(status), int(limit_us), _stream(stream)),
            "lmh_watchdog_selftest")
+
+
+def lmhead_bwd_dw_acc(dlogits: torch.Tensor, X: torch.Tensor, dW: torch.Tensor,
+                      status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dW[V,K] (FP32) += dlogits[M,V]^T . X[M,K]."""
+    _contig(dlogits, X, dW)
+    M, V = dlogits.shape
+    K = X.shape[1]
+    assert X.shape[0] == M and tuple(dW.shape) == (V, K) and dW.dtype == torch.float32
+    _check(lib().lmhead_bwd_dw_acc(_ptr(dlogits), _ptr(X), _ptr(dW), M, K, V, _ptr(status),
+                                   _stream(stream)), "lmhead_bwd_dw_acc")
+    return dW

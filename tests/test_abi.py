@@ -126,3 +126,11 @@ def test_fused_ce_workspace_size_and_validation():
         lmhead.LMH_ERR_INVALID_ARG
     assert f(A, A, A, A, A, P(0x10008), need, 16, 64, 64, -100, NULL, NULL) == \
         lmhead.LMH_ERR_MISALIGNED
+
+
+def test_dw_accumulate_validation():
+    f = lmhead.lib().lmhead_bwd_dw_acc
+    assert f(NULL, A, A, 16, 64, 64, NULL, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert f(A, A, A, 16, 60, 64, NULL, NULL) == lmhead.LMH_ERR_MISALIGNED
+    assert f(A, A, A, 16, 64, 60, NULL, NULL) == lmhead.LMH_ERR_MISALIGNED
+    assert f(A, A, P(0x10002), 16, 64, 64, NULL, NULL) == lmhead.LMH_ERR_MISALIGNED

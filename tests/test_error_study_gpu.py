@@ -1,0 +1,69 @@
+"""Error versus reduction width: FP32-output logits against BF16-output logits
+of the same kernel, both against the FP64 oracle.
+
+Megatron-LM PR #6252 "Add mixed-precision (FP32) LM output logits", "What
+does this PR do?": keeping the FP32 accumulator as the GEMM output, instead
+of rounding every logit to BF16, reduces the error at every reduction width
+tested; the widths and shapes are those of the page's "Method" (16 x K
+activations, 32768 x K vocabulary weights, K = 512 ... 16384), here with
+N(0,1) activations and N(0, 0.02^2) weights instead of integers (integers
+would make both outputs exact).  Run with -s to print the table.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lm_head_fp32_b200 import lmhead, synth
+from helpers import bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+K_WIDTHS = (512, 1024, 2048, 4096, 8192, 16384)
+
+
+def _loss64(L, t):
+    """Per-row cross-entropy of FP64 logits, plain definition."""
+    m = L.max(axis=1, keepdims=True)
+    lse = m[:, 0] + np.log(np.exp(L - m).sum(axis=1))
+    return lse - L[np.arange(L.shape[0]), t]
+
+
+def test_fp32_output_reduces_error_at_every_width():
+    M, V = 16, 32768
+    rows = []
+    for K in K_WIDTHS:
+        X = synth.normal_bf16((M, K), 1.0, 1234)
+        W = synth.normal_bf16((V, K), 0.02, 1235)
+        t = synth.targets(M, V, 0.0, 1234).numpy()
+        Xd, Wd = X.to(DEV), W.to(DEV)
+        l32 = torch.empty((M, V), dtype=torch.float32, device=DEV)
+        l16 = torch.empty((M, V), dtype=torch.bfloat16, device=DEV)
+        st = torch.zeros(1, dtype=torch.int32, device=DEV)
+        lmhead.lmhead_fwd(Xd, Wd, l32, st)
+        lmhead.lmhead_fwd(Xd, Wd, l16, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        ref = oracle.logits(bits(X), bits(W))
+        e32 = np.abs(l32.cpu().double().numpy() - ref)
+        e16 = np.abs(l16.float().cpu().double().numpy() - ref)
+        scale = float(np.sqrt((ref ** 2).mean()))
+        loss_ref = _loss64(ref, t)
+        dl32 = np.abs(_loss64(l32.cpu().double().numpy(), t) - loss_ref)
+        dl16 = np.abs(_loss64(l16.float().cpu().double().numpy(), t) - loss_ref)
+        tol = 1e-5 * math.sqrt(K) * float(X.float().abs().max()) * float(W.float().abs().max())
+        rows.append((K, scale, e32.max(), e16.max(), math.sqrt((e32 ** 2).mean()),
+                     math.sqrt((e16 ** 2).mean()), dl32.max(), dl16.max(), tol))
+    print("\n   K   rms(logit)  max|err| f32  max|err| bf16  rms err f32  rms err bf16  "
+          "max|dloss| f32  max|dloss| bf16")
+    for r in rows:
+        print(f"{r[0]:6d}  {r[1]:9.4f}  {r[2]:12.3e}  {r[3]:13.3e}  {r[4]:11.3e}  {r[5]:12.3e}  "
+              f"{r[6]:14.3e}  {r[7]:15.3e}")
+    for K, scale, m32, m16, r32, r16, d32, d16, tol in rows:
+        # the page's claim at this width: the FP32 output's error is materially
+        # (here: at least ten times) smaller, in the logits and in the loss
+        assert m32 * 10 < m16 and r32 * 10 < r16 and d32 * 10 < d16, K
+        # and the FP32 output meets the accumulation tolerance
+        assert m32 <= tol, K

@@ -160,3 +160,45 @@ def test_direct_store_epilogue_on_unaligned_output(dtype):
         assert int(st.item()) == 0
         assert torch.equal(out, expect)
         assert bool((buf[:off] == 0).all()) and bool((buf[off + n:] == 0).all()), "wrote outside"
+
+
+@pytest.mark.parametrize("M,K,V", [(300, 264, 1000), (17, 72, 40), (1024, 128, 4096)])
+def test_dw_accumulate_integer_exact(M, K, V):
+    """dW += dl^T X: with integer operands and an integer starting dW the sum is
+    exact, so the result equals dW0 + the exact product word for word, and
+    accumulating twice adds the product twice."""
+    dl = synth.int_bf16((M, V), 81 + M)
+    X = synth.int_bf16((M, K), 82 + K)
+    dW0 = torch.randint(-1000, 1001, (V, K), generator=torch.Generator().manual_seed(83)).float()
+    prod = torch.from_numpy(oracle.dw(bits(dl), bits(X))).float()
+    dW = dW0.to(DEV)
+    st = status_word()
+    lmhead.lmhead_bwd_dw_acc(dl.to(DEV), X.to(DEV), dW, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(dW.cpu(), dW0 + prod)
+    lmhead.lmhead_bwd_dw_acc(dl.to(DEV), X.to(DEV), dW, st)
+    torch.cuda.synchronize()
+    assert torch.equal(dW.cpu(), dW0 + 2 * prod)
+
+
+def test_dw_accumulate_random_both_epilogue_paths():
+    M, K, V = 200, 1000, 136
+    dl = synth.normal_bf16((M, V), 1e-3, 91)
+    X = synth.normal_bf16((M, K), 1.0, 92)
+    dW0 = (torch.randn((V, K), generator=torch.Generator().manual_seed(93)) * 1e-3).float()
+    ref = dW0.double().numpy() + oracle.dw(bits(dl), bits(X))
+    dld, Xd = dl.to(DEV), X.to(DEV)
+    a = dW0.to(DEV)
+    lmhead.lmhead_bwd_dw_acc(dld, Xd, a)
+    # an output a tensor map cannot describe takes the per-element atomic path
+    buf = torch.zeros(V * K + 1, dtype=torch.float32, device=DEV)
+    b = buf[1:].view(V, K)
+    b.copy_(dW0.to(DEV))
+    assert b.data_ptr() % 16 != 0
+    lmhead.lmhead_bwd_dw_acc(dld, Xd, b)
+    torch.cuda.synchronize()
+    tol = gemm_tol(M, dl, X) + 2.0 ** -23 * float(np.abs(ref).max())
+    assert_abs_close(a.cpu().double().numpy(), ref, tol, "dW accumulated")
+    assert torch.equal(a, b)
+    assert float(buf[0]) == 0.0
