@@ -169,6 +169,41 @@ LMH_API lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, const i
                                            int64_t V, int64_t ignore_index, int32_t *status,
                                            lmh_stream_t stream);
 
+/* Vocabulary-parallel cross-entropy (the vocabulary split across devices, as
+ * Megatron's VocabParallelCrossEntropy does, named in [P2] "Description").
+ * Device r holds logits[M, V_r] for vocabulary entries [offset_r, offset_r +
+ * V_r) of a vocabulary of vocab_total; targets are global ids.  The three
+ * calls below are the per-device parts; the exchange between devices (an
+ * all-gather of the [M,4] shard records) is the caller's.
+ *
+ * ce_fwd_shard: per row of this shard, shard_stats[M,4] = {m_r, d_r, x_y or 0,
+ *   1 if the target is in this shard else 0}; ignored rows (target ==
+ *   ignore_index) and bad targets (outside [0, vocab_total)) give zeros, bad
+ *   targets also set LMH_DEV_BAD_TARGET.
+ *   Requirements: 0 <= vocab_offset, vocab_offset + V <= vocab_total. */
+LMH_API lmh_status_t ce_fwd_shard(const float *logits, const int64_t *target, float *shard_stats,
+                                  int64_t M, int64_t V, int64_t vocab_offset, int64_t vocab_total,
+                                  int64_t ignore_index, int32_t *status, lmh_stream_t stream);
+
+/* ce_merge_shards: stats[M,4] = {m, d, x_y, loss} of the whole vocabulary
+ * from the num_shards records of every shard, laid out shard-major
+ * (shard_stats[r][M][4]): m = max_r m_r, d = sum_r d_r exp(m_r - m) taken in
+ * shard order (deterministic), x_y from the owning shard,
+ * loss = (m - x_y) + log d.  The result is what ce_fwd gives on the whole
+ * rows, up to the order of the sums. */
+LMH_API lmh_status_t ce_merge_shards(const float *shard_stats, int64_t num_shards,
+                                     const int64_t *target, float *stats, int64_t M,
+                                     int64_t vocab_total, int64_t ignore_index, int32_t *status,
+                                     lmh_stream_t stream);
+
+/* ce_bwd_shard: ce_bwd on a shard, with the merged stats: dl[i,j] =
+ * (exp(x_ij - m_i) / d_i - [vocab_offset + j == target_i]) * g_i. */
+LMH_API lmh_status_t ce_bwd_shard(const float *logits, const int64_t *target, const float *stats,
+                                  const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
+                                  int32_t dl_dtype, int64_t M, int64_t V, int64_t vocab_offset,
+                                  int64_t vocab_total, int64_t ignore_index, int32_t *status,
+                                  lmh_stream_t stream);
+
 /* dX = dlogits . W, the input gradient of logits = X . W^T
  * ([P1] "What does this PR do?", backward under the GEMM contract).
  *   dlogits [M,V] BF16.  W [V,K] BF16.

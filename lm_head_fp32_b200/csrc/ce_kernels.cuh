@@ -113,19 +113,25 @@ __device__ __forceinline__ int row_kind(int64_t y, int64_t V, int64_t ignore_ind
 }
 
 // stats[row] = {m, d, x_y, loss}.  VEC: V % 4 == 0 and logits 16-byte aligned.
-template <bool VEC, int THREADS = 512>
+// The rows hold vocabulary entries [voff, voff + V) of a vocabulary of Vtot
+// (voff = 0, Vtot = V for a whole row); targets are global ids.  SHARD: the
+// rows are one shard of a vocabulary split across devices, and the record is
+// {m, d, x_y or 0, 1 if the target lies in this shard else 0} for
+// ce_merge_shards_kernel to combine.
+template <bool VEC, int THREADS = 512, bool SHARD = false>
 __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict__ logits,
                                                             const int64_t *__restrict__ target,
                                                             float4 *__restrict__ stats, int64_t M,
                                                             int64_t V, int64_t ignore_index,
-                                                            int32_t *status)
+                                                            int32_t *status, int64_t voff,
+                                                            int64_t Vtot)
 {
     __shared__ MaxSum red[32];
     pdl_wait();  // the logits may come from the kernel just before this one
     pdl_launch_dependents();
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
         const int64_t y = target[row];
-        const int kind = row_kind(y, V, ignore_index);
+        const int kind = row_kind(y, Vtot, ignore_index);
         if (kind != 0) {
             if (threadIdx.x == 0) {
                 stats[row] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -160,11 +166,16 @@ __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict
         }
         s = block_merge(s, red);
         if (threadIdx.x == 0) {
-            const float xy = x[y];
-            // (m - x_y) first: exact when x_y is the maximum, so a near-zero
-            // loss is not swamped by the rounding of m + log(d).
-            const float loss = (s.m - xy) + logf(s.d);
-            stats[row] = make_float4(s.m, s.d, xy, loss);
+            if (SHARD) {
+                const bool owner = y >= voff && y < voff + V;
+                stats[row] = make_float4(s.m, s.d, owner ? x[y - voff] : 0.f, owner ? 1.f : 0.f);
+            } else {
+                const float xy = x[y];
+                // (m - x_y) first: exact when x_y is the maximum, so a near-zero
+                // loss is not swamped by the rounding of m + log(d).
+                const float loss = (s.m - xy) + logf(s.d);
+                stats[row] = make_float4(s.m, s.d, xy, loss);
+            }
         }
     }
 }
@@ -198,11 +209,13 @@ __device__ __forceinline__ void store1(__nv_bfloat16 *p, float a) { *p = __float
 // Each element is read before it is written, by the same thread, so dl may
 // alias logits when OutT is float (ALIAS: coherent loads instead of the
 // read-only path).
+// The rows hold vocabulary entries [voff, voff + V) of a vocabulary of Vtot
+// (a shard when voff > 0 or V < Vtot): the one-hot is at the global target.
 template <typename OutT, bool VEC, bool ALIAS, int THREADS = 512>
 __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
     const float *logits, const int64_t *__restrict__ target, const float4 *__restrict__ stats,
     const float *__restrict__ grad_loss, int64_t grad_stride, OutT *dl, int64_t M, int64_t V,
-    int64_t ignore_index, int32_t *status)
+    int64_t ignore_index, int32_t *status, int64_t voff, int64_t Vtot)
 {
     pdl_wait();
     pdl_launch_dependents();
@@ -210,8 +223,9 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
     // ones most likely still in L2
     for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
         const int64_t row = M - 1 - r;
-        const int64_t y = target[row];
-        const int kind = row_kind(y, V, ignore_index);
+        const int64_t yg = target[row];
+        const int kind = row_kind(yg, Vtot, ignore_index);
+        const int64_t y = yg - voff;  // local column of the target (may lie outside [0, V))
         const float *x = logits + row * V;
         OutT *o = dl + row * V;
         if (kind != 0) {
@@ -263,6 +277,37 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
                 store1(o + j, (exp_neg(v - m) * inv_d - (j == y)) * g);
             }
         }
+    }
+}
+
+// stats[i] = {m, d, x_y, loss} from R shard records (ce_fwd_kernel with
+// SHARD) laid out shard-major, shard_stats[r * M + i]: the pairs are merged
+// in shard order and x_y comes from the shard that owns the target.
+__global__ void __launch_bounds__(256)
+    ce_merge_shards_kernel(const float4 *__restrict__ shard_stats, int64_t R,
+                           const int64_t *__restrict__ target, float4 *__restrict__ stats, int64_t M,
+                           int64_t Vtot, int64_t ignore_index, int32_t *status)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < M;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int kind = row_kind(target[i], Vtot, ignore_index);
+        if (kind != 0) {
+            stats[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kind == 2 && status)
+                atomicOr(status, 1);
+            continue;
+        }
+        MaxSum s{-INFINITY, 0.f};
+        float xy = 0.f;
+        for (int64_t r = 0; r < R; ++r) {
+            const float4 q = shard_stats[r * M + i];
+            s = merge(s, MaxSum{q.x, q.y});
+            if (q.w != 0.f)
+                xy = q.z;
+        }
+        stats[i] = make_float4(s.m, s.d, xy, (s.m - xy) + logf(s.d));
     }
 }
 

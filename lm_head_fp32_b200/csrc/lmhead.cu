@@ -551,15 +551,20 @@ lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *stats, in
     float4 *st4 = reinterpret_cast<float4 *>(stats);
     if (vec)
         return launch_ex(lmh::ce_fwd_kernel<true, kCeThreads>, dim3(grid), dim3(kCeThreads), 0, s, 1u,
-                         logits, target, st4, M, V, ignore_index, status);
+                         logits, target, st4, M, V, ignore_index, status, int64_t{0}, V);
     return launch_ex(lmh::ce_fwd_kernel<false, kCeThreads>, dim3(grid), dim3(kCeThreads), 0, s, 1u,
-                     logits, target, st4, M, V, ignore_index, status);
+                     logits, target, st4, M, V, ignore_index, status, int64_t{0}, V);
 }
 
-lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *stats,
-                    const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
-                    int32_t dl_dtype, int64_t M, int64_t V, int64_t ignore_index,
-                    int32_t *status, lmh_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// ce_bwd over vocabulary entries [voff, voff + V) of a vocabulary of Vtot.
+lmh_status_t ce_bwd_range(const float *logits, const int64_t *target, const float *stats,
+                          const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
+                          int32_t dl_dtype, int64_t M, int64_t V, int64_t voff, int64_t Vtot,
+                          int64_t ignore_index, int32_t *status, lmh_stream_t stream)
 {
     if (!logits || !target || !stats || !grad_loss || !dlogits || M < 1 || V < 1 ||
         M > kMaxDim || V > kMaxDim)
@@ -584,14 +589,75 @@ lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *sta
                      : (alias ? lmh::ce_bwd_kernel<float, false, true, kCeThreads>
                               : lmh::ce_bwd_kernel<float, false, false, kCeThreads>);
         return launch_ex(k, dim3(grid), dim3(kCeThreads), 0, s, 1u, logits, target, st4, grad_loss,
-                         grad_loss_stride, o, M, V, ignore_index, status);
+                         grad_loss_stride, o, M, V, ignore_index, status, voff, Vtot);
     }
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(dlogits);
     const bool vec = (V % 4 == 0) && aligned(logits, 16) && aligned(o, 8);
     auto k = vec ? lmh::ce_bwd_kernel<__nv_bfloat16, true, false, kCeThreads>
                  : lmh::ce_bwd_kernel<__nv_bfloat16, false, false, kCeThreads>;
     return launch_ex(k, dim3(grid), dim3(kCeThreads), 0, s, 1u, logits, target, st4, grad_loss,
-                     grad_loss_stride, o, M, V, ignore_index, status);
+                     grad_loss_stride, o, M, V, ignore_index, status, voff, Vtot);
+}
+
+}  // namespace
+
+extern "C" {
+
+lmh_status_t ce_bwd(const float *logits, const int64_t *target, const float *stats,
+                    const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
+                    int32_t dl_dtype, int64_t M, int64_t V, int64_t ignore_index,
+                    int32_t *status, lmh_stream_t stream)
+{
+    return ce_bwd_range(logits, target, stats, grad_loss, grad_loss_stride, dlogits, dl_dtype, M, V,
+                        0, V, ignore_index, status, stream);
+}
+
+lmh_status_t ce_fwd_shard(const float *logits, const int64_t *target, float *shard_stats,
+                          int64_t M, int64_t V, int64_t vocab_offset, int64_t vocab_total,
+                          int64_t ignore_index, int32_t *status, lmh_stream_t stream)
+{
+    if (!logits || !target || !shard_stats || M < 1 || V < 1 || M > kMaxDim || V > kMaxDim ||
+        vocab_offset < 0 || vocab_total > kMaxDim || vocab_offset + V > vocab_total)
+        return LMH_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(target, 8) || !aligned(shard_stats, 16))
+        return LMH_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int grid = static_cast<int>(M);
+    float4 *st4 = reinterpret_cast<float4 *>(shard_stats);
+    if ((V % 4 == 0) && aligned(logits, 16))
+        return launch_ex(lmh::ce_fwd_kernel<true, kCeThreads, true>, dim3(grid), dim3(kCeThreads), 0,
+                         s, 1u, logits, target, st4, M, V, ignore_index, status, vocab_offset,
+                         vocab_total);
+    return launch_ex(lmh::ce_fwd_kernel<false, kCeThreads, true>, dim3(grid), dim3(kCeThreads), 0, s,
+                     1u, logits, target, st4, M, V, ignore_index, status, vocab_offset, vocab_total);
+}
+
+lmh_status_t ce_merge_shards(const float *shard_stats, int64_t num_shards, const int64_t *target,
+                             float *stats, int64_t M, int64_t vocab_total, int64_t ignore_index,
+                             int32_t *status, lmh_stream_t stream)
+{
+    if (!shard_stats || !target || !stats || num_shards < 1 || num_shards > 65536 || M < 1 ||
+        M > kMaxDim || vocab_total < 1 || vocab_total > kMaxDim)
+        return LMH_ERR_INVALID_ARG;
+    if (!aligned(shard_stats, 16) || !aligned(target, 8) || !aligned(stats, 16))
+        return LMH_ERR_MISALIGNED;
+    const int64_t blocks = (M + 255) / 256;
+    return launch_ex(lmh::ce_merge_shards_kernel, dim3(static_cast<unsigned>(blocks < 65535 ? blocks : 65535)),
+                     dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), 1u,
+                     reinterpret_cast<const float4 *>(shard_stats), num_shards, target,
+                     reinterpret_cast<float4 *>(stats), M, vocab_total, ignore_index, status);
+}
+
+lmh_status_t ce_bwd_shard(const float *logits, const int64_t *target, const float *stats,
+                          const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
+                          int32_t dl_dtype, int64_t M, int64_t V, int64_t vocab_offset,
+                          int64_t vocab_total, int64_t ignore_index, int32_t *status,
+                          lmh_stream_t stream)
+{
+    if (vocab_offset < 0 || vocab_total > kMaxDim || V < 1 || vocab_offset + V > vocab_total)
+        return LMH_ERR_INVALID_ARG;
+    return ce_bwd_range(logits, target, stats, grad_loss, grad_loss_stride, dlogits, dl_dtype, M, V,
+                        vocab_offset, vocab_total, ignore_index, status, stream);
 }
 
 }  // extern "C"

@@ -24,7 +24,7 @@ IGNORE_INDEX = -100
 
 EXPORTS = ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
            "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes", "lmhead_fwd_ce_noalloc",
-           "lmhead_bwd_dw_acc",
+           "lmhead_bwd_dw_acc", "ce_fwd_shard", "ce_merge_shards", "ce_bwd_shard",
            "lmh_status_string", "lmh_version", "lmh_watchdog_selftest")
 
 _lib = None
@@ -57,6 +57,11 @@ def lib() -> ctypes.CDLL:
         L.lmh_version.restype = ctypes.c_int32
         L.lmhead_fwd_ce.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P]
         L.lmhead_fwd_ce.restype = ctypes.c_int
+        L.ce_fwd_shard.argtypes = [P, P, P, I64, I64, I64, I64, I64, P, P]
+        L.ce_merge_shards.argtypes = [P, I64, P, P, I64, I64, I64, P, P]
+        L.ce_bwd_shard.argtypes = [P, P, P, P, I64, P, I32, I64, I64, I64, I64, I64, P, P]
+        for f in ("ce_fwd_shard", "ce_merge_shards", "ce_bwd_shard"):
+            getattr(L, f).restype = ctypes.c_int
         L.lmhead_bwd_dw_acc.argtypes = [P, P, P, I64, I64, I64, P, P]
         L.lmhead_bwd_dw_acc.restype = ctypes.c_int
         L.lmhead_fwd_ce_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
@@ -227,3 +232,44 @@ def lmhead_bwd_dw_acc(dlogits: torch.Tensor, X: torch.Tensor, dW: torch.Tensor,
     _check(lib().lmhead_bwd_dw_acc(_ptr(dlogits), _ptr(X), _ptr(dW), M, K, V, _ptr(status),
                                    _stream(stream)), "lmhead_bwd_dw_acc")
     return dW
+
+
+def ce_fwd_shard(logits: torch.Tensor, target: torch.Tensor, shard_stats: torch.Tensor,
+                 vocab_offset: int, vocab_total: int, ignore_index: int = IGNORE_INDEX,
+                 status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """shard_stats[M,4] = {m_r, d_r, x_y or 0, owner flag} of one vocabulary shard."""
+    _contig(logits, target, shard_stats)
+    M, V = logits.shape
+    assert tuple(shard_stats.shape) == (M, 4)
+    _check(lib().ce_fwd_shard(_ptr(logits), _ptr(target), _ptr(shard_stats), M, V,
+                              int(vocab_offset), int(vocab_total), int(ignore_index),
+                              _ptr(status), _stream(stream)), "ce_fwd_shard")
+    return shard_stats
+
+
+def ce_merge_shards(shard_stats: torch.Tensor, target: torch.Tensor, stats: torch.Tensor,
+                    vocab_total: int, ignore_index: int = IGNORE_INDEX,
+                    status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """stats[M,4] = {m, d, x_y, loss} from shard_stats[R,M,4] (shard-major)."""
+    _contig(shard_stats, target, stats)
+    R, M, four = shard_stats.shape
+    assert four == 4 and tuple(stats.shape) == (M, 4)
+    _check(lib().ce_merge_shards(_ptr(shard_stats), R, _ptr(target), _ptr(stats), M,
+                                 int(vocab_total), int(ignore_index), _ptr(status),
+                                 _stream(stream)), "ce_merge_shards")
+    return stats
+
+
+def ce_bwd_shard(logits: torch.Tensor, target: torch.Tensor, stats: torch.Tensor,
+                 grad_loss: torch.Tensor, dlogits: torch.Tensor, vocab_offset: int,
+                 vocab_total: int, ignore_index: int = IGNORE_INDEX,
+                 status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """ce_bwd on one vocabulary shard with the merged statistics."""
+    _contig(logits, target, stats, grad_loss, dlogits)
+    M, V = logits.shape
+    stride = 0 if grad_loss.numel() == 1 else 1
+    _check(lib().ce_bwd_shard(_ptr(logits), _ptr(target), _ptr(stats), _ptr(grad_loss), stride,
+                              _ptr(dlogits), _dtype_code(dlogits.dtype), M, V, int(vocab_offset),
+                              int(vocab_total), int(ignore_index), _ptr(status), _stream(stream)),
+           "ce_bwd_shard")
+    return dlogits
