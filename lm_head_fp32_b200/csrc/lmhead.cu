@@ -237,6 +237,11 @@ int pick_bn_tokens(int64_t M)
     return 256;
 }
 
+// L2 policy of W in the vocabulary GEMM: streamed once (evict first) when a
+// single token tile reads each W panel, normal when several token tiles reuse
+// it (measured: +13 % for M <= 128, -7 % at M = 1024 with evict first).
+int w_policy(int64_t M, int bn) { return M <= bn ? 1 : 0; }
+
 // CTA-pair tiles (256 x 256) are used when the n extent fills a 256-wide
 // tile.  LMH_GEMM_PAIR=0 or 1 in the environment forces single-CTA or pair
 // tiles where both are possible (a tuning aid; read once per process).
@@ -387,8 +392,8 @@ lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(K);
     p.m_fastest = 0;  // consecutive tiles share one W panel
-    p.l2_a = 1;       // W is streamed once (its panel's users run together)
-    p.l2_b = 2;       // X is reread by every tile
+    p.l2_a = w_policy(M, bn);
+    p.l2_b = 2;  // X is reread by every tile
     p.status = status;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, a, b, p, s)
@@ -520,7 +525,7 @@ lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target, 
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(K);
     p.m_fastest = 0;
-    p.l2_a = 1;
+    p.l2_a = w_policy(M, bn);
     p.l2_b = 2;
     p.status = status;
     p.ce_partial = static_cast<float2 *>(workspace);
@@ -736,7 +741,7 @@ extern "C" lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, cons
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(K);
     p.m_fastest = 0;
-    p.l2_a = 1;
+    p.l2_a = w_policy(M, bn);
     p.l2_b = 2;
     p.status = status;
     p.ce_partial = scratch;
