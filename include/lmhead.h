@@ -140,7 +140,7 @@ LMH_API lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *
                                    int64_t workspace_bytes, int64_t M, int64_t K, int64_t V,
                                    int64_t ignore_index, int32_t *status, lmh_stream_t stream);
 
-/* Scratch bytes lmhead_fwd_ce needs: M tokens x 8 * ceil(V / 256) slices x
+/* Scratch bytes lmhead_fwd_ce needs: 8 * ceil(V / 256) slices x M tokens x
  * 8 bytes (8 MB for M = 1024, V = 32768).  -1 for sizes out of range. */
 LMH_API int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V);
 

@@ -312,44 +312,46 @@ __global__ void __launch_bounds__(256)
 }
 
 // stats[i] = {m, d, x_y, loss} from the per-slice partials the fused
-// vocabulary GEMM wrote (partial[i * nslices + s]; the target logit is already
-// in stats[i].x_y).  One warp per token: lane l merges slices l, l + 32, ...
-// (eight 8-byte loads in flight), then the lanes are merged by a fixed
-// butterfly, so the result does not depend on scheduling.
+// vocabulary GEMM wrote (partial[s * M + i]; the target logit is already in
+// stats[i].x_y).  One CTA per 32 tokens, lane = token: warp w merges slices
+// w, w + WARPS, ... (each load is 32 consecutive tokens, eight in flight per
+// lane), then warp 0 merges the warps in order, so the result does not
+// depend on scheduling.
 template <int WARPS>
 __global__ void __launch_bounds__(WARPS * 32)
     ce_finalize_kernel(const float2 *__restrict__ partial, int64_t nslices,
                        const int64_t *__restrict__ target, float4 *stats, int64_t M, int64_t V,
                        int64_t ignore_index, int32_t *status)
 {
+    __shared__ MaxSum red[WARPS][32];
     pdl_wait();
     pdl_launch_dependents();
-    const int lane = threadIdx.x & 31;
-    const int64_t tok = static_cast<int64_t>(blockIdx.x) * WARPS + (threadIdx.x >> 5);
-    if (tok >= M)
-        return;  // whole warp
-    const float2 *row = partial + tok * nslices;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tok = static_cast<int64_t>(blockIdx.x) * 32 + lane;
     MaxSum s{-INFINITY, 0.f};
-    int64_t sl = lane;
-    for (; sl + 7 * 32 < nslices; sl += 8 * 32) {
-        float2 v[8];
+    if (tok < M) {
+        int64_t sl = warp;
+        for (; sl + 7 * WARPS < nslices; sl += 8 * WARPS) {
+            float2 v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            v[u] = row[sl + u * 32];
+            for (int u = 0; u < 8; ++u)
+                v[u] = partial[(sl + u * WARPS) * M + tok];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            s = merge(s, MaxSum{v[u].x, v[u].y});
+            for (int u = 0; u < 8; ++u)
+                s = merge(s, MaxSum{v[u].x, v[u].y});
+        }
+        for (; sl < nslices; sl += WARPS) {
+            const float2 v = partial[sl * M + tok];
+            s = merge(s, MaxSum{v.x, v.y});
+        }
     }
-    for (; sl < nslices; sl += 32) {
-        const float2 v = row[sl];
-        s = merge(s, MaxSum{v.x, v.y});
-    }
+    red[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0 && tok < M) {
+        MaxSum r = red[0][lane];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        MaxSum t{__shfl_xor_sync(0xffffffffu, s.m, o), __shfl_xor_sync(0xffffffffu, s.d, o)};
-        s = merge(s, t);
-    }
-    if (lane == 0) {
+        for (int w = 1; w < WARPS; ++w)
+            r = merge(r, red[w][lane]);
         const int64_t y = target[tok];
         const int kind = row_kind(y, V, ignore_index);
         if (kind != 0) {
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(WARPS * 32)
                 atomicOr(status, 1);
         } else {
             const float xy = reinterpret_cast<const float *>(stats)[tok * 4 + 2];
-            stats[tok] = make_float4(s.m, s.d, xy, (s.m - xy) + logf(s.d));
+            stats[tok] = make_float4(r.m, r.d, xy, (r.m - xy) + logf(r.d));
         }
     }
 }

@@ -55,11 +55,11 @@ struct GemmParams {
     int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
     int32_t l2_b;
     int32_t *status;
-    // fused cross-entropy statistics (vocabulary GEMM only): per token i and
-    // 32-wide vocabulary slice s, ce_partial[i * ce_nslices + s] = (max,
-    // sum-exp) of the slice; the target logit goes to ce_stats[4 i + 2].
+    // fused cross-entropy statistics (vocabulary GEMM only): per 32-wide
+    // vocabulary slice s and token i, ce_partial[s * Ndim + i] = (max,
+    // sum-exp) of the slice (a warp stores 32 consecutive tokens of one slice);
+    // the target logit goes to ce_stats[4 i + 2].
     float2 *ce_partial;
-    int64_t ce_nslices;
     const int64_t *ce_target;
     float *ce_stats;
 };
@@ -169,7 +169,7 @@ __device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int
                 dsum += exp_neg(rowp[col] - vmax);
         }
     }
-    p.ce_partial[static_cast<int64_t>(tok) * p.ce_nslices + slice] = make_float2(vmax, dsum);
+    p.ce_partial[slice * p.Ndim + tok] = make_float2(vmax, dsum);
     const int64_t y = p.ce_target[tok];
     if (y >= vbase && y < vbase + 32 && y < V)
         p.ce_stats[static_cast<int64_t>(tok) * 4 + 2] = rowp[y - vbase];

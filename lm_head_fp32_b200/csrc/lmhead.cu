@@ -278,7 +278,6 @@ lmh_status_t launch_gemm_ce(const Operand &a, const Operand &b, GemmParams p, in
                       static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
         return LMH_ERR_CUDA;
     *nslices = 4 * static_cast<int64_t>(C::CTAS) * ((p.Mdim + C::TILE_M - 1) / C::TILE_M);
-    p.ce_nslices = *nslices;
     return launch_gemm_impl<BN, false, false, float, true, PAIR, true>(ta, tb, tc, p, stream);
 }
 
@@ -535,8 +534,8 @@ lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target, 
     const lmh_status_t r = dispatch_ce(bn, a, b, p, &nslices, s);
     if (r != LMH_OK)
         return r;
-    constexpr int kFinalizeWarps = 8;  // tokens per CTA
-    const int64_t grid = (M + kFinalizeWarps - 1) / kFinalizeWarps;
+    constexpr int kFinalizeWarps = 32;  // 32 tokens per CTA, slices split over the warps
+    const int64_t grid = (M + 31) / 32;
     return launch_ex(lmh::ce_finalize_kernel<kFinalizeWarps>, dim3(static_cast<unsigned>(grid)),
                      dim3(kFinalizeWarps * 32), 0, s, 1u, static_cast<const float2 *>(workspace),
                      nslices, target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
@@ -751,8 +750,8 @@ extern "C" lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, cons
     const lmh_status_t r = dispatch_ce(bn, a, b, p, &nslices, s);
     if (r != LMH_OK)
         return r;
-    constexpr int kFinalizeWarps = 8;
-    const int64_t grid = (M + kFinalizeWarps - 1) / kFinalizeWarps;
+    constexpr int kFinalizeWarps = 32;
+    const int64_t grid = (M + 31) / 32;
     return launch_ex(lmh::ce_finalize_kernel<kFinalizeWarps>, dim3(static_cast<unsigned>(grid)),
                      dim3(kFinalizeWarps * 32), 0, s, 1u, static_cast<const float2 *>(scratch), nslices,
                      target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
