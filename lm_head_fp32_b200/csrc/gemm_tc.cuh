@@ -66,8 +66,12 @@ struct GemmParams {
 
 constexpr int kEpiWarps = 4;
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
+constexpr int kSmemPerSm = 233472;  // 228 KB per SM, of which 1 KB is reserved per CTA
 
-template <int BN, bool A_MN, bool B_MN, bool PAIR>
+// RES: CTAs meant to be resident per SM.  1 (persistent, deepest ring) for
+// the tensor-bound shapes; 2 for HBM-bound single-token-tile shapes, whose
+// tiles are then all in flight at once instead of running in waves.
+template <int BN, bool A_MN, bool B_MN, bool PAIR, int RES = 1>
 struct GemmCfg {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int TILE_M = kBlockM * CTAS;  // m extent of one (pair) tile
@@ -86,13 +90,15 @@ struct GemmCfg {
     static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_SLOT_BYTES;
     // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
     static constexpr int FIXED_BYTES = 1024 /* alignment slack */ + EPI_BYTES + 64 * 8;
-    static constexpr int STAGES_RAW = (kSmemLimit - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int BUDGET = RES == 1 ? kSmemLimit : kSmemPerSm / RES - 1024;
+    static constexpr int STAGES_RAW = (BUDGET - FIXED_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 16;
     static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
     static_assert(STAGES >= 2, "pipeline depth");
-    static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
+    static_assert(SMEM_BYTES <= BUDGET, "shared memory");
+    static_assert(RES * TMEM_COLS <= 512, "tensor memory of the resident CTAs");
 };
 
 template <int N>
@@ -188,12 +194,12 @@ __device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int
 // ACC (FP32 output): add the product to the output instead of overwriting it
 // (TMA reduce-add, or one atomic add per element on the direct path).
 template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
-          bool ACC = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+          bool ACC = false, int RES = 1>
+__global__ void __launch_bounds__(kGemmThreads, RES)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(

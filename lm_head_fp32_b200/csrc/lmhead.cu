@@ -169,12 +169,12 @@ bool make_operand_map(CUtensorMap *map, const Operand &op, uint32_t rows)
 
 // One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
 template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
-          bool ACC = false>
+          bool ACC = false, int RES = 1>
 lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                               GemmParams p, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
-    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE, ACC>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE, ACC, RES>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -184,6 +184,10 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
             cudaSuccess)
             return LMH_ERR_CUDA;
+        // several CTAs per SM need the whole unified memory as shared memory
+        if (RES > 1 && cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            100) != cudaSuccess)
+            return LMH_ERR_CUDA;
         attr_set.fetch_or(bit);
     }
     p.num_m_tiles = static_cast<int32_t>((p.Mdim + C::TILE_M - 1) / C::TILE_M);
@@ -191,24 +195,27 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
     const int64_t tiles = static_cast<int64_t>(p.num_m_tiles) * p.num_n_tiles;
     if (tiles > kMaxDim)
         return LMH_ERR_INVALID_ARG;
-    const int64_t units = num_sms() / C::CTAS;  // CTAs (or CTA pairs) resident at once
+    // persistent: one CTA (or CTA pair) per SM (pair); several resident per SM: one per tile
+    const int64_t units = RES == 1 ? num_sms() / C::CTAS : tiles;
     const int grid = static_cast<int>((tiles < units ? tiles : units) * C::CTAS);
     return launch_ex(kern, dim3(grid), dim3(lmh::kGemmThreads), C::SMEM_BYTES, stream,
                      PAIR ? 2u : 1u, ta, tb, tc, p);
 }
 
-template <int BN, bool A_MN, bool B_MN, typename OutT, bool PAIR>
+template <int BN, bool A_MN, bool B_MN, typename OutT, bool PAIR, int RES = 1>
 lmh_status_t launch_gemm(const Operand &a, const Operand &b, GemmParams p, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES>;
     CUtensorMap ta, tb, tc;
     if (!make_operand_map(&ta, a, lmh::kBlockM) || !make_operand_map(&tb, b, C::BN_CTA))
         return LMH_ERR_CUDA;
     if (make_out_map(&tc, p.out, sizeof(OutT) == 2, static_cast<uint64_t>(p.Mdim),
                      static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
-        return launch_gemm_impl<BN, A_MN, B_MN, OutT, true, PAIR>(ta, tb, tc, p, stream);
+        return launch_gemm_impl<BN, A_MN, B_MN, OutT, true, PAIR, false, false, RES>(ta, tb, tc, p,
+                                                                                   stream);
     std::memset(&tc, 0, sizeof tc);
-    return launch_gemm_impl<BN, A_MN, B_MN, OutT, false, PAIR>(ta, tb, tc, p, stream);
+    return launch_gemm_impl<BN, A_MN, B_MN, OutT, false, PAIR, false, false, RES>(ta, tb, tc, p,
+                                                                                stream);
 }
 
 // dW += dlogits^T . X (FP32): the dW GEMM with an accumulating epilogue.
@@ -267,28 +274,30 @@ bool use_pair(int bn, int64_t Mdim)
 // Vocabulary GEMM with the fused cross-entropy statistics (FP32 logits through
 // the TMA-store epilogue; the caller has checked that a tensor map can describe
 // them).  *nslices receives the number of 32-wide slices written.
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, int RES = 1>
 lmh_status_t launch_gemm_ce(const Operand &a, const Operand &b, GemmParams p, int64_t *nslices,
                             cudaStream_t stream)
 {
-    using C = GemmCfg<BN, false, false, PAIR>;
+    using C = GemmCfg<BN, false, false, PAIR, RES>;
     CUtensorMap ta, tb, tc;
     if (!make_operand_map(&ta, a, lmh::kBlockM) || !make_operand_map(&tb, b, C::BN_CTA) ||
         !make_out_map(&tc, p.out, false, static_cast<uint64_t>(p.Mdim),
                       static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
         return LMH_ERR_CUDA;
     *nslices = 4 * static_cast<int64_t>(C::CTAS) * ((p.Mdim + C::TILE_M - 1) / C::TILE_M);
-    return launch_gemm_impl<BN, false, false, float, true, PAIR, true>(ta, tb, tc, p, stream);
+    return launch_gemm_impl<BN, false, false, float, true, PAIR, true, false, RES>(ta, tb, tc, p,
+                                                                                 stream);
 }
 
 lmh_status_t dispatch_ce(int bn, const Operand &a, const Operand &b, GemmParams p, int64_t *nslices,
                          cudaStream_t s)
 {
+    // one token tile (bn covers every token): HBM-bound, two CTAs resident per SM
     switch (bn) {
-    case 16: return launch_gemm_ce<16, false>(a, b, p, nslices, s);
-    case 32: return launch_gemm_ce<32, false>(a, b, p, nslices, s);
-    case 64: return launch_gemm_ce<64, false>(a, b, p, nslices, s);
-    case 128: return launch_gemm_ce<128, false>(a, b, p, nslices, s);
+    case 16: return launch_gemm_ce<16, false, 2>(a, b, p, nslices, s);
+    case 32: return launch_gemm_ce<32, false, 2>(a, b, p, nslices, s);
+    case 64: return launch_gemm_ce<64, false, 2>(a, b, p, nslices, s);
+    case 128: return launch_gemm_ce<128, false, 2>(a, b, p, nslices, s);
     case 256:
         return use_pair(bn, p.Mdim) ? launch_gemm_ce<256, true>(a, b, p, nslices, s)
                                     : launch_gemm_ce<256, false>(a, b, p, nslices, s);
@@ -303,6 +312,17 @@ int64_t ce_slices(int64_t V) { return 8 * ((V + 255) / 256); }
 template <bool A_MN, bool B_MN, typename OutT>
 lmh_status_t dispatch_bn(int bn, const Operand &a, const Operand &b, GemmParams p, cudaStream_t s)
 {
+    if constexpr (!A_MN && !B_MN) {
+        // vocabulary GEMM with one token tile (bn covers every token): HBM-bound
+        // on W, so two CTAs resident per SM with one CTA per tile
+        switch (bn) {
+        case 16: return launch_gemm<16, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
+        case 32: return launch_gemm<32, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
+        case 64: return launch_gemm<64, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
+        case 128: return launch_gemm<128, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
+        default: break;
+        }
+    }
     if constexpr (!B_MN) {
         switch (bn) {
         case 16: return launch_gemm<16, A_MN, B_MN, OutT, false>(a, b, p, s);
