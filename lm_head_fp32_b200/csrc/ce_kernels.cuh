@@ -313,41 +313,59 @@ __global__ void __launch_bounds__(256)
 
 // stats[i] = {m, d, x_y, loss} from the per-slice partials the fused
 // vocabulary GEMM wrote (partial[s * M + i]; the target logit is already in
-// stats[i].x_y).  One CTA per 32 tokens, lane = token: warp w merges slices
-// w, w + WARPS, ... (each load is 32 consecutive tokens, eight in flight per
-// lane), then warp 0 merges the warps in order, so the result does not
+// stats[i].x_y).  One CTA per kFinalizeTokens = 8 tokens: lane = (slice
+// offset 0..3) x (token 0..7), so a warp-wide load reads four 64-byte runs of
+// eight consecutive tokens; warp w takes slice groups w, w + WARPS, ...
+// (eight loads in flight per lane).  The four lanes of a token are merged by
+// shuffles and the warps by warp 0 in a fixed order, so the result does not
 // depend on scheduling.
+constexpr int kFinalizeTokens = 8;
+
 template <int WARPS>
 __global__ void __launch_bounds__(WARPS * 32)
     ce_finalize_kernel(const float2 *__restrict__ partial, int64_t nslices,
                        const int64_t *__restrict__ target, float4 *stats, int64_t M, int64_t V,
                        int64_t ignore_index, int32_t *status)
 {
-    __shared__ MaxSum red[WARPS][32];
+    constexpr int T = kFinalizeTokens;
+    constexpr int SL = 32 / T;  // slices per warp-wide load
+    __shared__ MaxSum red[WARPS][T];
     pdl_wait();
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t tok = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+    const int64_t tok = static_cast<int64_t>(blockIdx.x) * T + (lane % T);
+    const int64_t sl0 = lane / T;
     MaxSum s{-INFINITY, 0.f};
     if (tok < M) {
-        int64_t sl = warp;
-        for (; sl + 7 * WARPS < nslices; sl += 8 * WARPS) {
+        int64_t g = warp;  // slice group: slices g * SL + sl0
+        for (; (g + 7 * WARPS) * SL < nslices; g += 8 * WARPS) {
             float2 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                v[u] = partial[(sl + u * WARPS) * M + tok];
+            for (int u = 0; u < 8; ++u) {
+                const int64_t sl = (g + u * WARPS) * SL + sl0;
+                v[u] = sl < nslices ? partial[sl * M + tok] : make_float2(-INFINITY, 0.f);
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 s = merge(s, MaxSum{v[u].x, v[u].y});
         }
-        for (; sl < nslices; sl += WARPS) {
-            const float2 v = partial[sl * M + tok];
-            s = merge(s, MaxSum{v.x, v.y});
+        for (; g * SL < nslices; g += WARPS) {
+            const int64_t sl = g * SL + sl0;
+            if (sl < nslices) {
+                const float2 v = partial[sl * M + tok];
+                s = merge(s, MaxSum{v.x, v.y});
+            }
         }
     }
-    red[warp][lane] = s;
+#pragma unroll
+    for (int off = T; off < 32; off <<= 1) {
+        const MaxSum o{__shfl_xor_sync(0xffffffffu, s.m, off), __shfl_xor_sync(0xffffffffu, s.d, off)};
+        s = merge(s, o);
+    }
+    if (lane < T)
+        red[warp][lane] = s;
     __syncthreads();
-    if (warp == 0 && tok < M) {
+    if (warp == 0 && lane < T && tok < M) {
         MaxSum r = red[0][lane];
 #pragma unroll
         for (int w = 1; w < WARPS; ++w)

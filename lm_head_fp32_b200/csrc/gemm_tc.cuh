@@ -15,17 +15,22 @@
 // contiguous dimension, so each epilogue warp stores 32 consecutive elements
 // (one 128-byte line for FP32) per instruction straight from registers.
 //
-// CTA roles (192 threads, one CTA per SM, persistent over output tiles):
+// CTA roles (64 + 32 EW threads, one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: fills a STAGES-deep ring of A/B k-blocks
 //   warp 1      tensor-memory owner and MMA issuer (one elected thread)
-//   warps 2..5  epilogue: tensor memory -> registers -> shared memory -> TMA
-//               bulk tensor store (or, for outputs a tensor map cannot
-//               describe, registers -> global stores)
+//   warps 2..   EW = 4 or 8 epilogue warps: tensor memory -> registers ->
+//               shared memory -> TMA bulk tensor store (or, for outputs a
+//               tensor map cannot describe, registers -> global stores).  A
+//               warp may only read its own quarter (warp % 4) of the 128
+//               tensor-memory lanes; with eight, two warps share each quarter
+//               and take alternate sub-tiles.
 // Two accumulators of BN columns let the epilogue of tile t overlap the MMAs
-// of tile t+1.  With the TMA-store epilogue each warp stages 32 x 32 sub-tiles
-// in two shared-memory slots and hands them to the TMA engine, so tensor
-// memory is released as soon as its values are in shared memory instead of
-// after 128 KB of global stores have drained.  Every wait is bounded (see
+// of tile t+1.  With the TMA-store epilogue the warps stage 32 x 32 sub-tiles
+// in eight shared-memory slots (two per warp, or one) and hand them to the TMA
+// engine, so tensor memory is released as soon as its values are in shared
+// memory instead of after 128 KB of global stores have drained.  Eight warps
+// halve the epilogue of a tile, which matters where no MMA hides it: the last
+// tile of each CTA when the fused cross-entropy statistics lengthen it.  Every wait is bounded (see
 // mbar_wait); on a timeout the CTA drains its own copies and MMAs, frees
 // tensor memory, sets a status bit and returns.
 #pragma once
@@ -38,7 +43,6 @@
 
 namespace lmh {
 
-constexpr int kGemmThreads = 192;
 constexpr int kBlockM = 128;  // MMA M: tensor-memory lanes
 constexpr int kBlockK = 64;   // one 128-byte swizzle row of BF16
 constexpr int kUmmaK = 16;    // K of one kind::f16 MMA
@@ -64,15 +68,26 @@ struct GemmParams {
     float *ce_stats;
 };
 
-constexpr int kEpiWarps = 4;
+constexpr int kEpiSlots = 8;  // 32 x EPI_CHUNK staging slots shared by the epilogue warps
+
+// Epilogue warps of each GEMM.  Measured at 1024 x 4096 x 32768 (L2 flushed,
+// medians): eight take the fused cross-entropy GEMM from 195.6 to 187.4 us,
+// where the statistics make the last tile's epilogue long; four are better
+// for the plain GEMMs (forward 170.0 against 172.1 us, dW 214.5 against
+// 223.3 us, dX equal), whose epilogue is short and whose extra store bursts
+// compete with the operand loads.
+constexpr int epi_warps(bool /*a_mn*/, bool /*b_mn*/, bool ce, bool /*acc*/) { return ce ? 8 : 4; }
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
 constexpr int kSmemPerSm = 233472;  // 228 KB per SM, of which 1 KB is reserved per CTA
 
 // RES: CTAs meant to be resident per SM.  1 (persistent, deepest ring) for
 // the tensor-bound shapes; 2 for HBM-bound single-token-tile shapes, whose
 // tiles are then all in flight at once instead of running in waves.
-template <int BN, bool A_MN, bool B_MN, bool PAIR, int RES = 1>
+template <int BN, bool A_MN, bool B_MN, bool PAIR, int RES = 1, int EW = 4>
 struct GemmCfg {
+    static_assert(EW == 4 || EW == 8, "epilogue warps");
+    static constexpr int THREADS = 64 + 32 * EW;
+    static constexpr int NSLOT = kEpiSlots / EW;  // staging slots per epilogue warp
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int TILE_M = kBlockM * CTAS;  // m extent of one (pair) tile
     static constexpr int BN_CTA = BN / CTAS;       // n rows of B held by each CTA
@@ -84,10 +99,10 @@ struct GemmCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
     static constexpr int EPI_CHUNK = BN < 32 ? BN : 32;  // accumulator columns per sub-tile
-    // two staging slots of 32 lanes x EPI_CHUNK columns per epilogue warp,
-    // sized for FP32 (a BF16 output uses half of each slot)
+    // staging slots of 32 lanes x EPI_CHUNK columns, sized for FP32 (a BF16
+    // output uses half of each)
     static constexpr int EPI_SLOT_BYTES = 32 * EPI_CHUNK * 4;
-    static constexpr int EPI_BYTES = kEpiWarps * 2 * EPI_SLOT_BYTES;
+    static constexpr int EPI_BYTES = kEpiSlots * EPI_SLOT_BYTES;
     // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
     static constexpr int FIXED_BYTES = 1024 /* alignment slack */ + EPI_BYTES + 64 * 8;
     static constexpr int BUDGET = RES == 1 ? kSmemLimit : kSmemPerSm / RES - 1024;
@@ -194,12 +209,12 @@ __device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int
 // ACC (FP32 output): add the product to the output instead of overwriting it
 // (TMA reduce-add, or one atomic add per element on the direct path).
 template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
-          bool ACC = false, int RES = 1>
-__global__ void __launch_bounds__(kGemmThreads, RES)
+          bool ACC = false, int RES = 1, int EW = epi_warps(A_MN, B_MN, CE, ACC)>
+__global__ void __launch_bounds__(64 + 32 * EW, RES)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES, EW>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -231,7 +246,7 @@ __global__ void __launch_bounds__(kGemmThreads, RES)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], kEpiWarps * C::CTAS);  // one arrival per epilogue warp
+            mbar_init(&acc_empty[a], EW * C::CTAS);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -396,15 +411,16 @@ __global__ void __launch_bounds__(kGemmThreads, RES)
             mbar_wait(drain, 0, &no_abort, kDrainLimitNs);
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 2..5)
-        const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+        // ------------------------------------------------ epilogue (warps 2 .. 2 + EW - 1)
+        const int q = warp & 3;            // tensor-memory lane quarter this warp may access
+        const int half = (warp - 2) >> 2;  // EW = 8: which alternate sub-tiles of the quarter
         const int row = q * 32 + lane;
         OutT *out = static_cast<OutT *>(p.out);
-        OutT *slots = reinterpret_cast<OutT *>(epi_smem + (warp - 2) * 2 * C::EPI_SLOT_BYTES);
+        OutT *slots = reinterpret_cast<OutT *>(epi_smem + (warp - 2) * C::NSLOT * C::EPI_SLOT_BYTES);
         constexpr int SLOT_ELEMS = C::EPI_SLOT_BYTES / static_cast<int>(sizeof(float));
+        uint32_t slot = 0;
         // where this warp releases an accumulator: the leader's barrier
         const uint32_t empty_addr0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
-        uint32_t slot = 0;
         uint32_t acc = 0, acc_phase = 0;
         for (int t = unit; t < num_tiles; t += num_units) {
             // every lane waits, then the warp agrees, so the .sync.aligned
@@ -421,17 +437,17 @@ __global__ void __launch_bounds__(kGemmThreads, RES)
             const bool m_ok = m < p.Mdim;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += C::EPI_CHUNK) {
+            for (int c = half * C::EPI_CHUNK; c < BN; c += (EW / 4) * C::EPI_CHUNK) {
                 if (TMA_STORE && n0 + c >= p.Ndim)
                     break;  // the rest of this tile lies beyond the output
                 uint32_t r[32];
                 tmem_ld_chunk<C::EPI_CHUNK>(taddr + c, r);
                 tmem_ld_wait();
                 if (TMA_STORE) {
-                    // slot is free once the store issued two sub-tiles ago
-                    // has finished reading it
+                    // the slot is free once the store issued NSLOT sub-tiles
+                    // ago has finished reading it
                     if (lane == 0)
-                        bulk_wait_read<1>();
+                        bulk_wait_read<C::NSLOT - 1>();
                     __syncwarp();
                     OutT *buf = slots + slot * SLOT_ELEMS;
 #pragma unroll
@@ -453,7 +469,7 @@ __global__ void __launch_bounds__(kGemmThreads, RES)
                         ce_subtile_stats(reinterpret_cast<const float *>(buf), lane, C::EPI_CHUNK,
                                          mbase + q * 32, p.Mdim, n0 + c + lane, p.Ndim, slice, p);
                     }
-                    slot ^= 1;
+                    slot = slot + 1 == C::NSLOT ? 0 : slot + 1;
                 } else if (m_ok) {
                     OutT *o = out + static_cast<int64_t>(n0 + c) * p.ldo + m;
 #pragma unroll

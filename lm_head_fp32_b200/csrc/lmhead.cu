@@ -169,12 +169,12 @@ bool make_operand_map(CUtensorMap *map, const Operand &op, uint32_t rows)
 
 // One GEMM launch: D[m,n] = sum_k A[m,k] B[n,k] -> out[n*ldo + m].
 template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
-          bool ACC = false, int RES = 1>
+          bool ACC = false, int RES = 1, int EW = lmh::epi_warps(A_MN, B_MN, CE, ACC)>
 lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                               GemmParams p, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES>;
-    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE, ACC, RES>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES, EW>;
+    auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE, ACC, RES, EW>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -198,7 +198,7 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
     // persistent: one CTA (or CTA pair) per SM (pair); several resident per SM: one per tile
     const int64_t units = RES == 1 ? num_sms() / C::CTAS : tiles;
     const int grid = static_cast<int>((tiles < units ? tiles : units) * C::CTAS);
-    return launch_ex(kern, dim3(grid), dim3(lmh::kGemmThreads), C::SMEM_BYTES, stream,
+    return launch_ex(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream,
                      PAIR ? 2u : 1u, ta, tb, tc, p);
 }
 
@@ -554,8 +554,8 @@ lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target, 
     const lmh_status_t r = dispatch_ce(bn, a, b, p, &nslices, s);
     if (r != LMH_OK)
         return r;
-    constexpr int kFinalizeWarps = 32;  // 32 tokens per CTA, slices split over the warps
-    const int64_t grid = (M + 31) / 32;
+    constexpr int kFinalizeWarps = 32;  // kFinalizeTokens tokens per CTA, slices split over the warps
+    const int64_t grid = (M + lmh::kFinalizeTokens - 1) / lmh::kFinalizeTokens;
     return launch_ex(lmh::ce_finalize_kernel<kFinalizeWarps>, dim3(static_cast<unsigned>(grid)),
                      dim3(kFinalizeWarps * 32), 0, s, 1u, static_cast<const float2 *>(workspace),
                      nslices, target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
@@ -771,7 +771,7 @@ extern "C" lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, cons
     if (r != LMH_OK)
         return r;
     constexpr int kFinalizeWarps = 32;
-    const int64_t grid = (M + 31) / 32;
+    const int64_t grid = (M + lmh::kFinalizeTokens - 1) / lmh::kFinalizeTokens;
     return launch_ex(lmh::ce_finalize_kernel<kFinalizeWarps>, dim3(static_cast<unsigned>(grid)),
                      dim3(kFinalizeWarps * 32), 0, s, 1u, static_cast<const float2 *>(scratch), nslices,
                      target, reinterpret_cast<float4 *>(stats), M, V, ignore_index, status);
