@@ -45,7 +45,8 @@ METRIC = "LM-head+CE fwd+bwd tokens/s; GEMM TFLOP/s and CE GB/s as % of B200 pea
 WORKLOAD = dict(name="lmhead_1024x4096x32768", M=1024, K=4096, V=32768)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("lm_head_fp32_b200/csrc/gemm_tc.cuh", "lm_head_fp32_b200/csrc/ce_kernels.cuh",
-                  "lm_head_fp32_b200/csrc/ptx.cuh", "lm_head_fp32_b200/csrc/lmhead.cu")
+                  "lm_head_fp32_b200/csrc/ptx.cuh", "lm_head_fp32_b200/csrc/lmhead.cu",
+                  "lm_head_fp32_b200/csrc/softmax_merge.cuh")
 FLUSH_BYTES = 512 << 20
 
 
@@ -82,10 +83,11 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def committed_traffic():
-    """Per-launch DRAM bytes of each kernel from the committed ncu summary, or
-    {} when that summary was taken on different kernel sources."""
-    p = os.path.join(ROOT, "profiles", "traffic_lmhead_1024x4096x32768.md")
+def committed_traffic(workload: str):
+    """Per-launch DRAM bytes of each kernel from the committed ncu summary of
+    this workload, or {} when there is none or it was taken on different
+    kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{workload}.md")
     if not os.path.exists(p):
         return {}
     txt = open(p).read()
@@ -400,7 +402,7 @@ def run_ours(args, cfg):
             "ce_fwd": ("hbm", ce_fwd_bytes),
             "ce_bwd": ("hbm", ce_bwd_bytes), "lmhead_bwd_dx": ("tensor", flop),
             "lmhead_bwd_dw": ("tensor", flop)}
-    traffic = committed_traffic()
+    traffic = committed_traffic(cfg.name)
     kernels = {}
     for j, n in enumerate(names):
         ms = statistics.mean(per_call[j])
@@ -510,7 +512,7 @@ def run_ce(args):
                        "l2": "inputs (5 GB) larger than L2"},
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["achieved"],
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kernels[dom]["frac"],
-                         "peak_source": f"{peak_src} (copy)", "traffic": committed_traffic().get(dom)},
+                         "peak_source": f"{peak_src} (copy)", "traffic": committed_traffic(cfg.name).get(dom)},
             "kernels": kernels, "gpu_launches": len(calls) * steps, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
