@@ -68,8 +68,8 @@ struct GemmParams {
     float *ce_stats;
 };
 
-constexpr int kEpiSlots = 8;
-constexpr unsigned kDwStorePaceNs = 200;  // pause after each dW sub-tile store  // 32 x EPI_CHUNK staging slots shared by the epilogue warps
+constexpr int kEpiSlots = 8;  // 32 x EPI_CHUNK staging slots shared by the epilogue warps
+constexpr unsigned kDwStorePaceNs = 200;  // pause after each dW sub-tile store
 
 // Epilogue warps of each GEMM.  Measured at 1024 x 4096 x 32768 (L2 flushed,
 // medians): eight take the fused cross-entropy GEMM from 195.6 to 187.4 us,
