@@ -121,7 +121,7 @@ LMH_API lmh_status_t ce_bwd(const float *logits, const int64_t *target, const fl
 
 /* logits = X . W^T (FP32) and the cross-entropy forward statistics of those
  * logits in one pass over them: the vocabulary GEMM's epilogue reduces every
- * 32-wide vocabulary slice of each token row to a partial (max, sum-exp) in
+ * 128-wide vocabulary block of each token row to a partial (max, sum-exp) in
  * `workspace` and records the target logit while the tile is still on chip,
  * and a second kernel merges each token's partials (in a fixed order) into
  * stats[M,4] = {m, d, x_y, loss}.  The logits are written but not read back
@@ -140,8 +140,8 @@ LMH_API lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *
                                    int64_t workspace_bytes, int64_t M, int64_t K, int64_t V,
                                    int64_t ignore_index, int32_t *status, lmh_stream_t stream);
 
-/* Scratch bytes lmhead_fwd_ce needs: 8 * ceil(V / 256) slices x M tokens x
- * 8 bytes (8 MB for M = 1024, V = 32768).  -1 for sizes out of range. */
+/* Scratch bytes lmhead_fwd_ce needs: 2 * ceil(V / 256) blocks x M tokens x
+ * 8 bytes (2 MB for M = 1024, V = 32768).  -1 for sizes out of range. */
 LMH_API int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V);
 
 /* lmhead_fwd_ce for callers that cannot allocate device memory (no
@@ -153,7 +153,7 @@ LMH_API int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V);
  * partial statistics in a fixed 8 MiB array inside the library, which every
  * GPU that loads the library holds until the process exits.  It allocates
  * nothing and calls no allocating routine.
- *   Limit: M * 8 * ceil(V / 256) <= 1048576 (e.g. M = 1024 with V up to
+ *   Limit: M * 2 * ceil(V / 256) <= 1048576 (e.g. M = 4096 with V up to
  *   32768); larger problems return LMH_ERR_INVALID_ARG before anything is
  *   launched.  (When V % 4 != 0 or logits is not 16-byte aligned the call
  *   runs lmhead_fwd then ce_fwd, which need no scratch, at any size.)

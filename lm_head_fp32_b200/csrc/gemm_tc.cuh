@@ -59,10 +59,11 @@ struct GemmParams {
     int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
     int32_t l2_b;
     int32_t *status;
-    // fused cross-entropy statistics (vocabulary GEMM only): per 32-wide
-    // vocabulary slice s and token i, ce_partial[s * Ndim + i] = (max,
-    // sum-exp) of the slice (a warp stores 32 consecutive tokens of one slice);
-    // the target logit goes to ce_stats[4 i + 2].
+    // fused cross-entropy statistics (vocabulary GEMM only): per 128-wide
+    // vocabulary block s (one CTA's rows of a tile) and token i,
+    // ce_partial[s * Ndim + i] = (max, sum-exp) of the block (a warp stores
+    // 32 consecutive tokens of one block); the target logit goes to
+    // ce_stats[4 i + 2].
     float2 *ce_partial;
     const int64_t *ce_target;
     float *ce_stats;
@@ -84,9 +85,10 @@ constexpr int kSmemPerSm = 233472;  // 228 KB per SM, of which 1 KB is reserved 
 // RES: CTAs meant to be resident per SM.  1 (persistent, deepest ring) for
 // the tensor-bound shapes; 2 for HBM-bound single-token-tile shapes, whose
 // tiles are then all in flight at once instead of running in waves.
-template <int BN, bool A_MN, bool B_MN, bool PAIR, int RES = 1, int EW = 4>
+template <int BN, bool A_MN, bool B_MN, bool PAIR, int RES = 1, int EW = 4, bool CE = false>
 struct GemmCfg {
     static_assert(EW == 4 || EW == 8, "epilogue warps");
+    static_assert(!CE || EW == 8, "the statistics exchange is laid out for eight epilogue warps");
     static constexpr int THREADS = 64 + 32 * EW;
     static constexpr int NSLOT = kEpiSlots / EW;  // staging slots per epilogue warp
     static constexpr int CTAS = PAIR ? 2 : 1;
@@ -104,13 +106,19 @@ struct GemmCfg {
     // output uses half of each)
     static constexpr int EPI_SLOT_BYTES = 32 * EPI_CHUNK * 4;
     static constexpr int EPI_BYTES = kEpiSlots * EPI_SLOT_BYTES;
-    // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
-    static constexpr int FIXED_BYTES = 1024 /* alignment slack */ + EPI_BYTES + 64 * 8;
+    // CE: per half of the epilogue warps, the (max, sum-exp) pairs of three
+    // lane quarters for the fourth to merge, and a full / free barrier pair
+    static constexpr int XCH_BYTES = CE ? 2 * 3 * 32 * 8 + 4 * 8 : 0;
+    // 1024 bytes of alignment slack, the ring (each stage with its full and
+    // empty barrier), the staging slots, acc_full[2], acc_empty[2], drain,
+    // the tensor-memory address and abort flag (16), the CE exchange
     static constexpr int BUDGET = RES == 1 ? kSmemLimit : kSmemPerSm / RES - 1024;
-    static constexpr int STAGES_RAW = (BUDGET - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES_RAW =
+        (BUDGET - 1024 - EPI_BYTES - 5 * 8 - 16 - XCH_BYTES) / (STAGE_BYTES + 16);
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 16;
+    static constexpr int SMEM_BYTES =
+        1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 16 + XCH_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
     static_assert(STAGES >= 2, "pipeline depth");
     static_assert(SMEM_BYTES <= BUDGET, "shared memory");
@@ -162,17 +170,16 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt,
 
 // Partial cross-entropy statistics of one staged sub-tile (FP32 logits):
 // lane l takes token row l of the 32 x 32 box in shared memory (32 vocabulary
-// columns starting at vbase; columns at or past V excluded), reduces it to
-// (max, sum of exp(x - max)) and stores it for slice `slice`; the lane whose
-// row holds its token's target column also records the target logit.  The
-// columns are visited in a lane-rotated order, so the 32 lanes read 32
-// different banks.
-__device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int rows, int vbase,
-                                                 int V, int tok, int ntok, int64_t slice,
-                                                 const GemmParams &p)
+// columns starting at vbase; columns at or past V excluded) and returns its
+// (max, sum of exp(x - max)); the lane whose row holds its token's target
+// column also records the target logit.  Lanes without a token return the
+// empty pair.  The columns are visited in a lane-rotated order, so the 32
+// lanes read 32 different banks.
+__device__ __forceinline__ MaxSum ce_subtile_stats(const float *buf, int lane, int rows, int vbase,
+                                                   int V, int tok, int ntok, const GemmParams &p)
 {
     if (lane >= rows || tok >= ntok)
-        return;
+        return MaxSum{-INFINITY, 0.f};
     const float *rowp = buf + lane * 32;
     const int nvalid = V - vbase;  // may be <= 0 (a slice past the vocabulary) or > 32
     float vmax = -INFINITY;
@@ -191,10 +198,10 @@ __device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int
                 dsum += exp_neg(rowp[col] - vmax);
         }
     }
-    p.ce_partial[slice * p.Ndim + tok] = make_float2(vmax, dsum);
     const int64_t y = p.ce_target[tok];
     if (y >= vbase && y < vbase + 32 && y < V)
         p.ce_stats[static_cast<int64_t>(tok) * 4 + 2] = rowp[y - vbase];
+    return MaxSum{vmax, dsum};
 }
 
 // TMA_STORE: the output is written through tmC, a tensor map over
@@ -204,9 +211,13 @@ __device__ __forceinline__ void ce_subtile_stats(const float *buf, int lane, int
 // rows of B, the leader (rank 0) issues the MMAs, and each CTA's tensor
 // memory receives its 128 rows of the accumulator.  B is read from L2 once
 // per pair instead of once per SM.
-// CE (vocabulary GEMM, FP32 output, TMA_STORE): also emit the partial
-// cross-entropy statistics of every 32-wide vocabulary slice (see
-// ce_subtile_stats), so that the logits need not be read back.
+// CE (vocabulary GEMM, FP32 output, TMA_STORE, eight epilogue warps): also
+// emit the partial cross-entropy statistics of every CTA's 128-wide
+// vocabulary block, so that the logits need not be read back.  Each warp
+// reduces its lane quarter of a sub-tile (ce_subtile_stats); the four warps
+// of a half hand their pairs to the one on quarter 0 through shared memory
+// (two mbarriers, bounded waits), which merges them in quarter order and
+// stores one pair per token.
 // ACC (FP32 output): add the product to the output instead of overwriting it
 // (TMA reduce-add, or one atomic add per element on the direct path).
 template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR, bool CE = false,
@@ -215,7 +226,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES, EW>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES, EW, CE>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -230,6 +241,11 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
     uint64_t *drain = bars + 2 * S + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // CE exchange: xch_full[2], xch_free[2], then xch[2][3][32] pairs
+    uint64_t *xch_full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(bars) +
+                                                      C::BAR_BYTES + 16);
+    uint64_t *xch_free = xch_full + 2;
+    MaxSum *xch = reinterpret_cast<MaxSum *>(xch_free + 2);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -250,6 +266,12 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
             mbar_init(&acc_empty[a], EW * C::CTAS);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
+        if (CE) {
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(&xch_full[h], 3);  // the warps on lane quarters 1..3
+                mbar_init(&xch_free[h], 1);  // the warp on quarter 0, once it has read them
+            }
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -420,6 +442,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
         OutT *slots = reinterpret_cast<OutT *>(epi_smem + (warp - 2) * C::NSLOT * C::EPI_SLOT_BYTES);
         constexpr int SLOT_ELEMS = C::EPI_SLOT_BYTES / static_cast<int>(sizeof(float));
         uint32_t slot = 0;
+        uint32_t xch_phase = 0;
         // where this warp releases an accumulator: the leader's barrier
         const uint32_t empty_addr0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
         uint32_t acc = 0, acc_phase = 0;
@@ -472,10 +495,34 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                     }
                     if constexpr (CE) {
                         // the TMA store only reads the slot, so it can be read here too
-                        const int64_t slice =
-                            static_cast<int64_t>(mt * C::CTAS + static_cast<int>(rank)) * 4 + q;
-                        ce_subtile_stats(reinterpret_cast<const float *>(buf), lane, C::EPI_CHUNK,
-                                         mbase + q * 32, p.Mdim, n0 + c + lane, p.Ndim, slice, p);
+                        const int tok = n0 + c + lane;
+                        const MaxSum sv =
+                            ce_subtile_stats(reinterpret_cast<const float *>(buf), lane,
+                                             C::EPI_CHUNK, mbase + q * 32, p.Mdim, tok, p.Ndim, p);
+                        MaxSum *xh = xch + half * 3 * 32;
+                        if (q != 0) {
+                            if (mbar_wait(&xch_free[half], xch_phase ^ 1, abort_flag))
+                                xh[(q - 1) * 32 + lane] = sv;
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive(&xch_full[half]);
+                        } else {
+                            const bool got = mbar_wait(&xch_full[half], xch_phase, abort_flag);
+                            MaxSum r = sv;
+                            if (got) {
+#pragma unroll
+                                for (int j = 0; j < 3; ++j)
+                                    r = merge(r, xh[j * 32 + lane]);
+                            }
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive(&xch_free[half]);
+                            if (got && lane < C::EPI_CHUNK && tok < p.Ndim) {
+                                const int64_t block = mt * C::CTAS + static_cast<int>(rank);
+                                p.ce_partial[block * p.Ndim + tok] = make_float2(r.m, r.d);
+                            }
+                        }
+                        xch_phase ^= 1;
                     }
                     slot = slot + 1 == C::NSLOT ? 0 : slot + 1;
                 } else if (m_ok) {

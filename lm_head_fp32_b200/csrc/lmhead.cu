@@ -173,7 +173,7 @@ template <int BN, bool A_MN, bool B_MN, typename OutT, bool TMA_STORE, bool PAIR
 lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                               GemmParams p, cudaStream_t stream)
 {
-    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES, EW>;
+    using C = GemmCfg<BN, A_MN, B_MN, PAIR, RES, EW, CE>;
     auto kern = lmh::gemm_tc_kernel<BN, A_MN, B_MN, OutT, TMA_STORE, PAIR, CE, ACC, RES, EW>;
     // set once per process and device; the attribute is per function
     static std::atomic<uint64_t> attr_set{0};
@@ -273,7 +273,7 @@ bool use_pair(int bn, int64_t Mdim)
 
 // Vocabulary GEMM with the fused cross-entropy statistics (FP32 logits through
 // the TMA-store epilogue; the caller has checked that a tensor map can describe
-// them).  *nslices receives the number of 32-wide slices written.
+// them).  *nslices receives the number of 128-wide vocabulary blocks written.
 template <int BN, bool PAIR, int RES = 1>
 lmh_status_t launch_gemm_ce(const Operand &a, const Operand &b, GemmParams p, int64_t *nslices,
                             cudaStream_t stream)
@@ -284,7 +284,7 @@ lmh_status_t launch_gemm_ce(const Operand &a, const Operand &b, GemmParams p, in
         !make_out_map(&tc, p.out, false, static_cast<uint64_t>(p.Mdim),
                       static_cast<uint64_t>(p.Ndim), static_cast<uint64_t>(p.ldo), C::EPI_CHUNK))
         return LMH_ERR_CUDA;
-    *nslices = 4 * static_cast<int64_t>(C::CTAS) * ((p.Mdim + C::TILE_M - 1) / C::TILE_M);
+    *nslices = static_cast<int64_t>(C::CTAS) * ((p.Mdim + C::TILE_M - 1) / C::TILE_M);
     return launch_gemm_impl<BN, false, false, float, true, PAIR, true, false, RES>(ta, tb, tc, p,
                                                                                  stream);
 }
@@ -305,9 +305,10 @@ lmh_status_t dispatch_ce(int bn, const Operand &a, const Operand &b, GemmParams 
     }
 }
 
-// Slices of partial statistics the fused GEMM may write for a vocabulary of V
-// (both tile modes fit: 8 per 256 vocabulary columns).
-int64_t ce_slices(int64_t V) { return 8 * ((V + 255) / 256); }
+// Blocks of partial statistics the fused GEMM may write for a vocabulary of V
+// (one per CTA's 128 rows of a tile; both tile modes fit: 2 per 256
+// vocabulary columns).
+int64_t ce_slices(int64_t V) { return 2 * ((V + 255) / 256); }
 
 template <bool A_MN, bool B_MN, typename OutT>
 lmh_status_t dispatch_bn(int bn, const Operand &a, const Operand &b, GemmParams p, cudaStream_t s)

@@ -179,7 +179,7 @@ def lmhead_fwd_ce_noalloc(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor
                           stream=None):
     """lmhead_fwd_ce without a workspace, for callers that cannot allocate
     device memory: the partial statistics live in a fixed 8 MiB array inside
-    the library (M * 8 * ceil(V/256) <= 1048576).  Calls that overlap on the
+    the library (M * 2 * ceil(V/256) <= 1048576).  Calls that overlap on the
     GPU share that array and race."""
     _contig(X, W, target, logits, stats)
     M, K = X.shape

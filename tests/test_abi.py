@@ -111,8 +111,9 @@ def test_watchdog_selftest_validation():
 
 def test_fused_ce_workspace_size_and_validation():
     L = lmhead.lib()
-    assert lmhead.lmhead_fwd_ce_workspace_bytes(1024, 32768) == 8 * 128 * 1024 * 8
-    assert lmhead.lmhead_fwd_ce_workspace_bytes(16, 1) == 8 * 1 * 16 * 8
+    # two 128-wide vocabulary blocks per 256 columns, one (max, sum-exp) pair each per token
+    assert lmhead.lmhead_fwd_ce_workspace_bytes(1024, 32768) == 2 * 128 * 1024 * 8
+    assert lmhead.lmhead_fwd_ce_workspace_bytes(16, 1) == 2 * 1 * 16 * 8
     assert lmhead.lmhead_fwd_ce_workspace_bytes(0, 10) == -1
     f = L.lmhead_fwd_ce
     need = lmhead.lmhead_fwd_ce_workspace_bytes(16, 64)

@@ -46,8 +46,8 @@ def _without_allocation(X, W, t):
 
 
 def test_no_alloc_matches_workspace_entry_point_twice():
-    # the largest problem the fixed array holds at this vocabulary: M * 8 * ceil(V/256) = 2^20
-    M, K, V = 1024, 256, 32768
+    # the largest problem the fixed array holds at this vocabulary: M * 2 * ceil(V/256) = 2^20
+    M, K, V = 4096, 256, 32768
     for seed in (301, 302):
         X, W, t = _inputs(seed, M, K, V)
         l_ref, s_ref, st_ref = _with_workspace(X, W, t)
@@ -62,7 +62,7 @@ def test_no_alloc_matches_workspace_entry_point_twice():
 
 
 def test_no_alloc_rejects_problems_beyond_its_array():
-    M, K, V = 1025, 64, 32768          # one token more than the array holds
+    M, K, V = 4097, 64, 32768          # one token more than the array holds
     X, W, t = _inputs(303, M, K, V)
     logits = torch.empty((M, V), dtype=torch.float32, device=DEV)
     stats = torch.empty((M, 4), dtype=torch.float32, device=DEV)
