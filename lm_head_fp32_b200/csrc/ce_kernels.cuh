@@ -141,6 +141,13 @@ __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict
             continue;  // uniform across the block: no barrier skipped unevenly
         }
         const float *x = logits + row * V;
+        // the target logit is fetched up front by the thread that reports the
+        // row, so its latency hides behind the row's stream
+        const int64_t yl = y - voff;  // local column (may lie outside [0, V) for a shard)
+        const bool owner = yl >= 0 && yl < V;
+        float xy = 0.f;
+        if (threadIdx.x == 0 && owner)
+            xy = x[yl];
         MaxSum s{-INFINITY, 0.f};
         if (VEC) {
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
@@ -167,10 +174,8 @@ __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict
         s = block_merge(s, red);
         if (threadIdx.x == 0) {
             if (SHARD) {
-                const bool owner = y >= voff && y < voff + V;
-                stats[row] = make_float4(s.m, s.d, owner ? x[y - voff] : 0.f, owner ? 1.f : 0.f);
+                stats[row] = make_float4(s.m, s.d, xy, owner ? 1.f : 0.f);
             } else {
-                const float xy = x[y];
                 // (m - x_y) first: exact when x_y is the maximum, so a near-zero
                 // loss is not swamped by the rounding of m + log(d).
                 const float loss = (s.m - xy) + logf(s.d);
@@ -228,6 +233,9 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
         const int64_t y = yg - voff;  // local column of the target (may lie outside [0, V))
         const float *x = logits + row * V;
         OutT *o = dl + row * V;
+        // issued before the branch so that their latency overlaps the target's
+        const float4 st = stats[row];
+        const float g = grad_loss[row * grad_stride];
         if (kind != 0) {
             if (kind == 2 && status && threadIdx.x == 0)
                 atomicOr(status, 1);
@@ -240,10 +248,8 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
             }
             continue;
         }
-        const float4 st = stats[row];
         const float m = st.x;
         const float inv_d = 1.0f / st.y;
-        const float g = grad_loss[row * grad_stride];
         if (VEC) {
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
             const int64_t n4 = V >> 2;
