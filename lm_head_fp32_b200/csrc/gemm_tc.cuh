@@ -30,9 +30,9 @@
 // engine, so tensor memory is released as soon as its values are in shared
 // memory instead of after 128 KB of global stores have drained.  Eight warps
 // halve the epilogue of a tile, which matters where no MMA hides it: the last
-// tile of each CTA when the fused cross-entropy statistics lengthen it.  Every wait is bounded (see
-// mbar_wait); on a timeout the CTA drains its own copies and MMAs, frees
-// tensor memory, sets a status bit and returns.
+// tile of each CTA when the fused cross-entropy statistics lengthen it.
+// Every wait is bounded (see mbar_wait); on a timeout the CTA drains its own
+// copies and MMAs, frees tensor memory, sets a status bit and returns.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
