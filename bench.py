@@ -226,7 +226,9 @@ def run_reference(args):
     g = cfg.grad_scalar(t)
     import numpy as np
     import oracle
-    per_step = max(1, min(args.cpu_sample, 16))
+    # tokens per step sized so that the whole run stays near a minute and a
+    # half of host time (about 0.1 s per token on 16 cores), 1 to 16 tokens
+    per_step = max(1, min(args.cpu_sample, 16, 900 // max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_step(X, W, t, g, np.arange(per_step, dtype=np.int64) + (i * per_step) % cfg.M)
     t0 = time.perf_counter()
