@@ -6,12 +6,14 @@ W ~ N(0,0.02^2) in BF16, 2% of targets ignored, grad_loss = 1/num_valid).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload lmhead_1024x4096x32768 | lmhead_4096x4096x128256 |
-                                ce_8192x151936_outliers | sweep]
+                                ce_8192x151936_outliers | sweep | bitexact_16x512x32768]
 
 The default workload is the one the metric is quoted on.  The other LM-head
 workload and the wide-row cross-entropy workload print the same kind of line;
 "sweep" runs the FP32-versus-BF16 output comparison of the GEMM (15 shapes,
-N = 32768, 10 warm-up pairs, 30 alternating-order samples, medians).
+N = 32768, 10 warm-up pairs, 30 alternating-order samples, medians);
+"bitexact_16x512x32768" times the latency-bound smoke workload (lmhead_fwd,
+ce_fwd, ce_bwd) in microseconds.
 
 Prints one JSON line on rank 0.  Timing: CUDA events on the launching stream
 around every step (and every call inside it), L2 flushed by a 512 MiB write
@@ -64,7 +66,7 @@ def parse():
                          "statistics in one pass) then ce_bwd, dX, dW")
     ap.add_argument("--workload", default="lmhead_1024x4096x32768",
                     choices=["lmhead_1024x4096x32768", "lmhead_4096x4096x128256",
-                             "ce_8192x151936_outliers", "sweep"])
+                             "ce_8192x151936_outliers", "sweep", "bitexact_16x512x32768"])
     return ap.parse_args()
 
 
@@ -601,6 +603,94 @@ def run_sweep(args):
         pg.destroy_process_group()
 
 
+def run_latency(args):
+    """The bit-exact smoke workload (16 x 512 x 32768, integer BF16 operands):
+    it fits in L2, so it is latency-bound and is reported in microseconds per
+    step of lmhead_fwd, ce_fwd and ce_bwd (BF16 gradient), replayed from a
+    CUDA graph (the eager step time and each call's eager time, means over
+    the timed steps, are given too), with no roofline fraction."""
+    import torch
+    from lm_head_fp32_b200 import lmhead, synth
+
+    world, rank, local, pg, dev = gpu_setup(args)
+    cfg = synth.BITEXACT
+    X, W, t = cfg.make()
+    Xd, Wd, td = X.to(dev), W.to(dev), t.to(dev)
+    M, V = cfg.M, cfg.V
+    g = torch.full((1,), cfg.grad_scalar(t), dtype=torch.float32, device=dev)
+    logits = torch.empty((M, V), dtype=torch.float32, device=dev)
+    stats = torch.empty((M, 4), dtype=torch.float32, device=dev)
+    dl = torch.empty((M, V), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["lmhead_fwd", "ce_fwd", "ce_bwd"]
+    calls = [lambda: lmhead.lmhead_fwd(Xd, Wd, logits, status),
+             lambda: lmhead.ce_fwd(logits, td, stats, -100, status),
+             lambda: lmhead.ce_bwd(logits, td, stats, g, dl, -100, status)]
+    for _ in range(max(args.warmup, 3)):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+          for _ in range(K_steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(pg)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)
+    for i in range(K_steps):
+        ev[i][0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            ev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(pg)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    per = {n: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_steps)) * 1e3
+           for j, n in enumerate(names)}
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(K_steps)]
+    eager_ms = max_over_ranks(sum(step_ms), pg, dev)
+
+    # the same step captured once in a CUDA graph and replayed K times: at this
+    # size the launches, not the kernels, set the step time
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph):
+            for c in calls:
+                c()
+    stream.wait_stream(side)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg)
+    a.record(stream)
+    for _ in range(K_steps):
+        graph.replay()
+    z.record(stream)
+    torch.cuda.synchronize()
+    total_ms = max_over_ranks(a.elapsed_time(z), pg, dev)
+    del graph
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    line = {"metric": "latency of lmhead_fwd + ce_fwd + ce_bwd (us per step, CUDA graph replay)",
+            "value": 1e3 * total_ms / K_steps, "unit": "us", "n_gpus": world, "steps": K_steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / K_steps, "higher_is_better": False,
+            "eager_us_per_step": 1e3 * eager_ms / K_steps,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "M": M, "K": cfg.K, "V": V, "operands": "BF16 integers",
+                       "l2": "inputs fit in L2 (latency-bound; no flush, no roofline fraction)"},
+            "kernels_us": {n: round(v, 2) for n, v in per.items()},
+            "gpu_launches": len(calls) * K_steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -609,6 +699,8 @@ def main():
     from lm_head_fp32_b200 import synth
     if args.workload == "sweep":
         run_sweep(args)
+    elif args.workload == "bitexact_16x512x32768":
+        run_latency(args)
     elif args.workload == "ce_8192x151936_outliers":
         run_ce(args)
     elif args.workload == "lmhead_4096x4096x128256":
