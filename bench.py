@@ -216,6 +216,13 @@ def cpu_baseline(cfg, X, W, t, g, tokens: int):
                       f"(logits, CE fwd, CE bwd, dX rows, their dW share), FP64, {dt:.1f} s"}
 
 
+def reference_tokens_per_step(steps: int, warmup: int, cap: int) -> int:
+    """Tokens of the oracle's sample per reference step: 1 to min(cap, 16),
+    sized so that the whole run stays near a minute and a half of host time
+    (about 0.1 s per token on 16 cores)."""
+    return max(1, min(cap, 16, 900 // max(1, steps + warmup)))
+
+
 def run_reference(args):
     world, rank, local, pg = dist_setup(args)
     if rank != 0:
@@ -228,9 +235,7 @@ def run_reference(args):
     g = cfg.grad_scalar(t)
     import numpy as np
     import oracle
-    # tokens per step sized so that the whole run stays near a minute and a
-    # half of host time (about 0.1 s per token on 16 cores), 1 to 16 tokens
-    per_step = max(1, min(args.cpu_sample, 16, 900 // max(1, args.steps + args.warmup)))
+    per_step = reference_tokens_per_step(args.steps, args.warmup, args.cpu_sample)
     for i in range(args.warmup):
         oracle_step(X, W, t, g, np.arange(per_step, dtype=np.int64) + (i * per_step) % cfg.M)
     t0 = time.perf_counter()
