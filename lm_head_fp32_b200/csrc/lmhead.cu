@@ -272,6 +272,19 @@ bool use_pair(int bn, int64_t Mdim)
     return o < 0 ? true : o == 1;
 }
 
+// The single-token-tile vocabulary GEMM (two CTAs per SM) in CTA pairs: each
+// CTA stages half of X, so X crosses L2 -> SM once per pair instead of once
+// per CTA.  It pays only when X is large (measured at V = 32768: 128 tokens,
+// K = 16384: 204.8 -> 190.5 us; K = 4096: 61.5 -> 63.5 us; 64 tokens: no
+// gain at any K).
+bool use_pair_small(int bn, int64_t Mdim, int64_t Kdim)
+{
+    if (bn != 128 || Kdim < 16384 || Mdim < 256)
+        return false;
+    const int o = pair_override();
+    return o < 0 ? true : o == 1;
+}
+
 // Vocabulary GEMM with the fused cross-entropy statistics (FP32 logits through
 // the TMA-store epilogue; the caller has checked that a tensor map can describe
 // them).  *nslices receives the number of 128-wide vocabulary blocks written.
@@ -298,7 +311,9 @@ lmh_status_t dispatch_ce(int bn, const Operand &a, const Operand &b, GemmParams 
     case 16: return launch_gemm_ce<16, false, 2>(a, b, p, nslices, s);
     case 32: return launch_gemm_ce<32, false, 2>(a, b, p, nslices, s);
     case 64: return launch_gemm_ce<64, false, 2>(a, b, p, nslices, s);
-    case 128: return launch_gemm_ce<128, false, 2>(a, b, p, nslices, s);
+    case 128:
+        return use_pair_small(bn, p.Mdim, p.Kdim) ? launch_gemm_ce<128, true, 2>(a, b, p, nslices, s)
+                                                  : launch_gemm_ce<128, false, 2>(a, b, p, nslices, s);
     case 256:
         return use_pair(bn, p.Mdim) ? launch_gemm_ce<256, true>(a, b, p, nslices, s)
                                     : launch_gemm_ce<256, false>(a, b, p, nslices, s);
@@ -321,7 +336,10 @@ lmh_status_t dispatch_bn(int bn, const Operand &a, const Operand &b, GemmParams 
         case 16: return launch_gemm<16, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
         case 32: return launch_gemm<32, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
         case 64: return launch_gemm<64, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
-        case 128: return launch_gemm<128, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
+        case 128:
+            return use_pair_small(bn, p.Mdim, p.Kdim)
+                       ? launch_gemm<128, A_MN, B_MN, OutT, true, 2>(a, b, p, s)
+                       : launch_gemm<128, A_MN, B_MN, OutT, false, 2>(a, b, p, s);
         default: break;
         }
     }

@@ -60,7 +60,7 @@ def check(X, W, t, ignore=-100, rows=None):
 @pytest.mark.parametrize("M,K,V", [(16, 512, 32768), (300, 264, 1000), (17, 72, 32776),
                                    (130, 1024, 520), (257, 136, 2052), (1, 8, 4),
                                    (64, 4096, 128256), (128, 1024, 8200),
-                                   (300, 136, 200), (140, 256, 252)])
+                                   (300, 136, 200), (140, 256, 252), (96, 16384, 520)])
 def test_fused_ce_matches_oracle(M, K, V):
     X = synth.normal_bf16((M, K), 1.0, 51 + M)
     W = synth.normal_bf16((V, K), 0.05, 52 + V)

@@ -71,7 +71,7 @@ def test_integer_exactness_k_sweep(golden_dir):
 
 @pytest.mark.parametrize("M,K,V", [(300, 1000, 1000), (17, 72, 32776), (130, 4096, 520),
                                    (1, 8, 1), (257, 136, 129), (1024, 256, 384),
-                                   (64, 520, 4104), (100, 1024, 8200)])
+                                   (64, 520, 4104), (100, 1024, 8200), (100, 16384, 1032)])
 def test_logits_random_ragged(M, K, V):
     X = synth.normal_bf16((M, K), 1.0, 11 + M)
     W = synth.normal_bf16((V, K), 0.02, 12 + V)
