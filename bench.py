@@ -1,15 +1,19 @@
 #!/usr/bin/env python
 """Benchmark of the LM-head loss path: one step = the five calls
 lmhead_fwd -> ce_fwd -> ce_bwd (BF16 dlogits) -> lmhead_bwd_dx -> lmhead_bwd_dw
-on one synthetic batch (M=1024 tokens, K=4096, V=32768; X ~ N(0,1),
-W ~ N(0,0.02^2) in BF16, 2% of targets ignored, grad_loss = 1/num_valid).
+on one synthetic batch (default: M=4096 tokens, K=4096, V=128256; X ~ N(0,1),
+W ~ N(0,0.02^2) in BF16, 1% of targets ignored, grad_loss = 1/num_valid; the
+FP32 logits take 2.1 GB).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload lmhead_1024x4096x32768 | lmhead_4096x4096x128256 |
-                                ce_8192x151936_outliers | sweep | bitexact_16x512x32768]
+                    [--workload lmhead_4096x4096x128256 | lmhead_1024x4096x32768 |
+                                lmhead_<M>x<K>x<V> | ce_8192x151936_outliers | sweep |
+                                bitexact_16x512x32768]
 
-The default workload is the one the metric is quoted on.  The other LM-head
-workload and the wide-row cross-entropy workload print the same kind of line;
+The default workload is the largest LM-head configuration of the method that
+fits one GPU.  The mid-size LM head (and any lmhead_<M>x<K>x<V> shape, N(0,1) x
+N(0,0.02^2) operands with 1% of rows ignored, used for scaled profiles) and the
+wide-row cross-entropy workload print the same kind of line;
 "sweep" runs the FP32-versus-BF16 output comparison of the GEMM (15 shapes,
 N = 32768, 10 warm-up pairs, 30 alternating-order samples, medians);
 "bitexact_16x512x32768" times the latency-bound smoke workload (lmhead_fwd,
@@ -44,12 +48,21 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LM-head+CE fwd+bwd tokens/s; GEMM TFLOP/s and CE GB/s as % of B200 peak"
-WORKLOAD = dict(name="lmhead_1024x4096x32768", M=1024, K=4096, V=32768)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("lm_head_fp32_b200/csrc/gemm_tc.cuh", "lm_head_fp32_b200/csrc/ce_kernels.cuh",
                   "lm_head_fp32_b200/csrc/ptx.cuh", "lm_head_fp32_b200/csrc/lmhead.cu",
                   "lm_head_fp32_b200/csrc/softmax_merge.cuh")
 FLUSH_BYTES = 512 << 20
+L2_NOTE = ("flushed between steps outside the timed events: a 512 MiB write, then a read of "
+           "it, so that no dirty line of the flush is left for the step to write back")
+
+
+def flush_l2(buf):
+    """Evict the L2 (126 MB) between timed steps: write a buffer four times
+    its size, then read it back, which also writes back the dirty lines of
+    the write before the next step starts."""
+    buf.zero_()
+    return buf.sum()
 
 
 def parse():
@@ -64,10 +77,41 @@ def parse():
     ap.add_argument("--step", choices=["separate", "fused"], default="separate",
                     help="separate: the five calls; fused: lmhead_fwd_ce (logits and CE "
                          "statistics in one pass) then ce_bwd, dX, dW")
-    ap.add_argument("--workload", default="lmhead_1024x4096x32768",
-                    choices=["lmhead_1024x4096x32768", "lmhead_4096x4096x128256",
-                             "ce_8192x151936_outliers", "sweep", "bitexact_16x512x32768"])
+    ap.add_argument("--parallel", choices=["replicas", "vocab"], default="replicas",
+                    help="N > 1: replicas = every rank runs its own batch (weak scaling); "
+                         "vocab = the vocabulary is split across the ranks, one batch in all "
+                         "(strong scaling; NCCL all-gather of the per-row records and "
+                         "all-reduce of dX)")
+    ap.add_argument("--workload", default="lmhead_4096x4096x128256", type=workload_name,
+                    help="lmhead_4096x4096x128256 (default), lmhead_1024x4096x32768, "
+                         "lmhead_<M>x<K>x<V>, ce_8192x151936_outliers, sweep, "
+                         "bitexact_16x512x32768")
     return ap.parse_args()
+
+
+FIXED_WORKLOADS = ("ce_8192x151936_outliers", "sweep", "bitexact_16x512x32768")
+_LMHEAD_RE = re.compile(r"lmhead_(\d+)x(\d+)x(\d+)$")
+
+
+def workload_name(name: str) -> str:
+    if name in FIXED_WORKLOADS or _LMHEAD_RE.match(name):
+        return name
+    raise argparse.ArgumentTypeError(f"unknown workload {name!r}")
+
+
+def lmhead_config(name: str):
+    """The LM-head workload of that name: the two named configurations keep
+    their own seeds and ignore fractions; any other lmhead_<M>x<K>x<V> draws
+    X ~ N(0,1), W ~ N(0,0.02^2) and ignores 1% of the rows."""
+    from lm_head_fp32_b200 import synth
+    for c in (synth.LARGEVOCAB, synth.MIDSIZE):
+        if c.name == name:
+            return c
+    m = _LMHEAD_RE.match(name)
+    if not m:
+        raise ValueError(f"not an LM-head workload: {name}")
+    M, K, V = (int(v) for v in m.groups())
+    return synth.GemmConfig(name, M, K, V, "normal", ignore_frac=0.01)
 
 
 def load_peaks():
@@ -216,11 +260,14 @@ def cpu_baseline(cfg, X, W, t, g, tokens: int):
                       f"(logits, CE fwd, CE bwd, dX rows, their dW share), FP64, {dt:.1f} s"}
 
 
-def reference_tokens_per_step(steps: int, warmup: int, cap: int) -> int:
+def reference_tokens_per_step(steps: int, warmup: int, cap: int, K: int = 4096,
+                              V: int = 32768) -> int:
     """Tokens of the oracle's sample per reference step: 1 to min(cap, 16),
     sized so that the whole run stays near a minute and a half of host time
-    (about 0.1 s per token on 16 cores)."""
-    return max(1, min(cap, 16, 900 // max(1, steps + warmup)))
+    (about 0.1 s per token on 16 cores at K = 4096, V = 32768; the cost of a
+    token grows with K * V)."""
+    budget = int(900 * (4096 * 32768) / (K * V))
+    return max(1, min(cap, 16, budget // max(1, steps + warmup)))
 
 
 def run_reference(args):
@@ -229,13 +276,13 @@ def run_reference(args):
         if pg is not None:
             pg.destroy_process_group()
         return
-    from lm_head_fp32_b200 import synth
-    cfg = synth.MIDSIZE
+    name = args.workload if _LMHEAD_RE.match(args.workload) else "lmhead_4096x4096x128256"
+    cfg = lmhead_config(name)
     X, W, t = cfg.make()
     g = cfg.grad_scalar(t)
     import numpy as np
     import oracle
-    per_step = reference_tokens_per_step(args.steps, args.warmup, args.cpu_sample)
+    per_step = reference_tokens_per_step(args.steps, args.warmup, args.cpu_sample, cfg.K, cfg.V)
     for i in range(args.warmup):
         oracle_step(X, W, t, g, np.arange(per_step, dtype=np.int64) + (i * per_step) % cfg.M)
     t0 = time.perf_counter()
@@ -320,7 +367,7 @@ def run_ours(args, cfg):
             c()
 
     for _ in range(max(args.warmup, 3)):
-        flush.zero_()
+        flush_l2(flush)
         step()
     torch.cuda.synchronize()
     assert int(status.item()) == 0, f"device status {int(status.item())}"
@@ -336,7 +383,7 @@ def run_ours(args, cfg):
     sampler.start()
     time.sleep(0.25)                      # let the sampler attach
     for i in range(K_steps):
-        flush.zero_()                     # L2 flush, outside the timed events
+        flush_l2(flush)                     # L2 flush, outside the timed events
         e = ev[i]
         e[0].record(stream)
         for j, c in enumerate(calls):
@@ -353,37 +400,51 @@ def run_ours(args, cfg):
     value = world * M * K_steps / (total_ms / 1e3)
 
     # end to end through the public API: every step copies its X and targets
-    # from pinned host memory and reads its per-row loss back.  Inputs are
-    # double-buffered and copied on a second stream, so step i+1's copy runs
-    # under step i's kernels, as in a training loop with a prefetching loader.
+    # from pinned host memory, and its per-row statistics (the loss) and dX
+    # (the gradient handed back to the layer below) to pinned host memory.
+    # Inputs and outputs are double-buffered; inputs are copied on one side
+    # stream and outputs on another, so step i+1's input copy and step i-1's
+    # output copy run under step i's kernels, as in a training loop with a
+    # prefetching loader.  dW stays on the device with W.
     Xh = X.pin_memory()
     th = t.pin_memory()
-    lossh = [torch.empty((M, 4), dtype=torch.float32).pin_memory() for _ in range(2)]
+    outh = [(torch.empty((M, 4), dtype=torch.float32).pin_memory(),
+             torch.empty((M, K), dtype=torch.float32).pin_memory()) for _ in range(2)]
     Xb = [Xd, torch.empty_like(Xd)]
     tb = [td, torch.empty_like(td)]
-    cs = torch.cuda.Stream(device=dev)
+    sb = [stats, torch.empty_like(stats)]
+    dXb = [dX, torch.empty_like(dX)]
+    h2d_s = torch.cuda.Stream(device=dev)
+    d2h_s = torch.cuda.Stream(device=dev)
     copied = [torch.cuda.Event() for _ in range(2)]
     done = [torch.cuda.Event() for _ in range(2)]
+    out_copied = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step(i):
         b = i % 2
         if i >= 2:
-            cs.wait_event(done[b])          # step i-2 has finished with buffer b
-        with torch.cuda.stream(cs):
+            h2d_s.wait_event(done[b])       # step i-2 has finished with input buffer b
+        with torch.cuda.stream(h2d_s):
             Xb[b].copy_(Xh, non_blocking=True)
             tb[b].copy_(th, non_blocking=True)
-            copied[b].record(cs)
+            copied[b].record(h2d_s)
         stream.wait_event(copied[b])
+        if i >= 2:
+            stream.wait_event(out_copied[b])  # step i-2's outputs have left buffer b
         if fused:
-            lmhead.lmhead_fwd_ce(Xb[b], Wd, tb[b], logits, stats, ws, -100, status)
+            lmhead.lmhead_fwd_ce(Xb[b], Wd, tb[b], logits, sb[b], ws, -100, status)
         else:
             lmhead.lmhead_fwd(Xb[b], Wd, logits, status)
-            lmhead.ce_fwd(logits, tb[b], stats, -100, status)
-        lmhead.ce_bwd(logits, tb[b], stats, gd, dl, -100, status)
-        lmhead.lmhead_bwd_dx(dl, Wd, dX, status)
+            lmhead.ce_fwd(logits, tb[b], sb[b], -100, status)
+        lmhead.ce_bwd(logits, tb[b], sb[b], gd, dl, -100, status)
+        lmhead.lmhead_bwd_dx(dl, Wd, dXb[b], status)
         lmhead.lmhead_bwd_dw(dl, Xb[b], dW, status)
-        lossh[b].copy_(stats, non_blocking=True)
         done[b].record(stream)
+        d2h_s.wait_event(done[b])
+        with torch.cuda.stream(d2h_s):
+            outh[b][0].copy_(sb[b], non_blocking=True)
+            outh[b][1].copy_(dXb[b], non_blocking=True)
+            out_copied[b].record(d2h_s)
 
     e2e_steps = max(10, min(K_steps, 100))
     for i in range(4):
@@ -391,15 +452,18 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    cs.wait_event(a)
+    h2d_s.wait_event(a)
+    d2h_s.wait_event(a)
     for i in range(e2e_steps):
         e2e_step(i)
+    for b in range(2):
+        stream.wait_event(out_copied[b])    # the last results are on the host
     z.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a.elapsed_time(z), pg, dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     h2d = Xh.numel() * Xh.element_size() + th.numel() * th.element_size()
-    d2h = lossh[0].numel() * lossh[0].element_size()
+    d2h = sum(o.numel() * o.element_size() for o in outh[0])
 
     # roofline of every kernel; the dominant one goes in "roofline"
     peaks, peak_src = load_peaks()
@@ -436,21 +500,156 @@ def run_ours(args, cfg):
             "config": {"workload": cfg.name, "M": M, "K": K, "V": V, "logits": "fp32",
                        "dlogits": "bf16", "dX_dW": "fp32", "accumulate": "fp32",
                        "ignored_rows": M - nv, "grad_loss": "1/num_valid",
-                       "l2": "flushed between steps (512 MiB write outside the timed events)",
+                       "l2": L2_NOTE,
                        "parallelism": f"replicas x{world}",
                        "step": ("lmhead_fwd_ce, ce_bwd, lmhead_bwd_dx, lmhead_bwd_dw" if fused else
                                 "lmhead_fwd, ce_fwd, ce_bwd, lmhead_bwd_dx, lmhead_bwd_dw")},
             "roofline": roofline, "kernels": kernels,
             "e2e": {"value": world * M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "note": "pinned-host inputs copied on a second stream, double-buffered; "
-                            "no L2 flush (the step's working set is far larger than L2)"},
+                    "note": "X and targets in, stats and dX out, pinned host memory, "
+                            "double-buffered on two side streams; no L2 flush (the step's "
+                            "working set is far larger than L2)"},
             "gpu_launches": sum(2 if n == "lmhead_fwd_ce" else 1 for n in names) * K_steps,
             "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of oracle work: the sample shrinks as the vocabulary grows
         sample = max(8, int(args.cpu_sample * 32768 * 4096 / (cfg.V * cfg.K)))
         line["cpu_baseline"] = cpu_baseline(cfg, X, W, t, g, sample)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def vocab_shard_inputs(cfg, world: int, rank: int):
+    """This rank's inputs of a vocabulary-parallel step: the whole batch (the
+    same X and targets on every rank) and rows [off, off + n) of W."""
+    from lm_head_fp32_b200 import vocab_parallel
+    X, W, t = cfg.make()
+    off, n = vocab_parallel.shard_bounds(cfg.V, world, rank)
+    return X, W[off:off + n].contiguous(), t, off, n
+
+
+def vocab_line(cfg, world: int, steps: int, warmup: int, total_ms: float, stage_ms: dict,
+               clocks, nv: int, peaks, peak_src: str, shard_rows: int) -> dict:
+    """The JSON line of a vocabulary-parallel run: every rank works on the same
+    M tokens, so the job processes M tokens per step whatever the rank count
+    (strong scaling); total_ms is the maximum over ranks of the summed step
+    times, stage_ms this rank's mean time per stage."""
+    M, K = cfg.M, cfg.K
+    flop = 2.0 * M * K * shard_rows
+    work = {"lmhead_fwd": ("tensor", flop), "lmhead_bwd_dx": ("tensor", flop),
+            "lmhead_bwd_dw": ("tensor", flop),
+            "ce_fwd_shard": ("hbm", nv * shard_rows * 4 + M * 24),
+            "ce_bwd_shard": ("hbm", nv * shard_rows * 4 + M * shard_rows * 2 + M * 24)}
+    kernels = {}
+    for n, ms in stage_ms.items():
+        if n not in work or ms <= 0:
+            kernels[n] = {"ms": round(ms, 5)}
+            continue
+        bound, w = work[n]
+        if bound == "tensor":
+            ach, peak, unit = w / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        else:
+            ach, peak, unit = w / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        kernels[n] = {"ms": round(ms, 5), "bound": bound, "achieved": round(ach, 1), "unit": unit,
+                      "frac": round(ach / peak, 4), "algorithmic": w}
+    dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["ms"])
+    kd = kernels[dom]
+    return {"metric": METRIC, "value": M * steps / (total_ms / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": total_ms / steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "M": M, "K": K, "V": cfg.V, "logits": "fp32",
+                       "dlogits": "bf16", "dX_dW": "fp32", "ignored_rows": M - nv,
+                       "grad_loss": "1/num_valid", "parallelism": f"vocab{world}",
+                       "nccl_ranks": world, "vocab_rows_per_rank": shard_rows,
+                       "l2": L2_NOTE,
+                       "step": "lmhead_fwd, ce_fwd_shard, all-gather [M,4], ce_merge_shards, "
+                               "ce_bwd_shard, lmhead_bwd_dx, all-reduce dX, lmhead_bwd_dw"},
+            "roofline": {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"],
+                         "peak": peaks["bf16_tflops"] if kd["bound"] == "tensor" else peaks["hbm_gbs"],
+                         "unit": kd["unit"], "frac": kd["frac"],
+                         "peak_source": f"{peak_src} (burst)", "traffic": None},
+            "kernels": kernels, "clocks": clocks}
+
+
+def run_vocab(args, cfg):
+    """Vocabulary-parallel step across the ranks (strong scaling)."""
+    import torch
+    from lm_head_fp32_b200 import vocab_parallel
+
+    world, rank, local, pg, dev = gpu_setup(args)
+    X, Ws, t, off, n = vocab_shard_inputs(cfg, world, rank)
+    g = cfg.grad_scalar(t)
+    Xd, Wd, td = X.to(dev), Ws.to(dev), t.to(dev)
+    gd = torch.tensor([g], dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        flush_l2(flush)
+        vocab_parallel.step(Xd, Wd, td, off, cfg.V, gd, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    stages = vocab_parallel.STAGES
+    ev = [{} for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(pg)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)
+    for i in range(args.steps):
+        flush_l2(flush)
+        starts[i].record(stream)
+
+        def mark(name, i=i):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev[i][name] = e
+        vocab_parallel.step(Xd, Wd, td, off, cfg.V, gd, status=status, mark=mark)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(pg)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    step_ms = [starts[i].elapsed_time(ev[i][stages[-1]]) for i in range(args.steps)]
+    total_ms = max_over_ranks(sum(step_ms), pg, dev)
+    stage_ms = {}
+    for j, s in enumerate(stages):
+        prev = [starts[i] if j == 0 else ev[i][stages[j - 1]] for i in range(args.steps)]
+        stage_ms[s] = statistics.mean(prev[i].elapsed_time(ev[i][s]) for i in range(args.steps))
+    peaks, peak_src = load_peaks()
+    nv = int((t != -100).sum())
+    line = vocab_line(cfg, world, args.steps, args.warmup, total_ms, stage_ms, clocks, nv, peaks,
+                      peak_src, n)
+    line["gpu_launches"] = (6 if n > 0 else 1) * args.steps
+
+    # end to end: every step copies X and the targets in from pinned host
+    # memory and the statistics and dX out, on the compute stream
+    Xh, th = X.pin_memory(), t.pin_memory()
+    sh = torch.empty((cfg.M, 4), dtype=torch.float32).pin_memory()
+    dxh = torch.empty((cfg.M, cfg.K), dtype=torch.float32).pin_memory()
+    e2e_steps = max(5, min(args.steps, 50))
+    barrier(pg)
+    torch.cuda.synchronize()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        Xd.copy_(Xh, non_blocking=True)
+        td.copy_(th, non_blocking=True)
+        stats, dX, _, _, _ = vocab_parallel.step(Xd, Wd, td, off, cfg.V, gd, status=status)
+        sh.copy_(stats, non_blocking=True)
+        dxh.copy_(dX, non_blocking=True)
+    z.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(z), pg, dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    line["e2e"] = {"value": cfg.M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": Xh.numel() * Xh.element_size() + th.numel() * 8,
+                   "d2h_bytes_per_step": sh.numel() * 4 + dxh.numel() * 4,
+                   "note": "copies on the compute stream, not overlapped"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -563,7 +762,7 @@ def run_sweep(args):
                "bf16": lambda: lmhead.lmhead_fwd(X, W, o16, status)}
 
         def sample(k):
-            flush.zero_()
+            flush_l2(flush)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             run[k]()
@@ -601,7 +800,8 @@ def run_sweep(args):
             "median_overhead_pct_K_ge_8192": statistics.median(ov8),
             "shapes_within_10pct": sum(1 for o in ov if o <= 10.0),
             "range_pct": [min(ov), max(ov)], "shapes": rows, "peak_source": peak_src,
-            "protocol": "10 warm-up pairs, 30 alternating-order samples, medians, L2 flushed"}
+            "protocol": "10 warm-up pairs, 30 alternating-order samples, medians, L2 flushed "
+                        "(512 MiB write then read) before every sample"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -701,17 +901,16 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    from lm_head_fp32_b200 import synth
     if args.workload == "sweep":
         run_sweep(args)
     elif args.workload == "bitexact_16x512x32768":
         run_latency(args)
     elif args.workload == "ce_8192x151936_outliers":
         run_ce(args)
-    elif args.workload == "lmhead_4096x4096x128256":
-        run_ours(args, synth.LARGEVOCAB)
+    elif args.parallel == "vocab":
+        run_vocab(args, lmhead_config(args.workload))
     else:
-        run_ours(args, synth.MIDSIZE)
+        run_ours(args, lmhead_config(args.workload))
 
 
 if __name__ == "__main__":

@@ -159,7 +159,10 @@ LMH_API int64_t lmhead_fwd_ce_workspace_bytes(int64_t M, int64_t V);
  *   runs lmhead_fwd then ce_fwd, which need no scratch, at any size.)
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept for the life of the
+ *   process: do not use this call on a device after cudaDeviceReset (or
+ *   after its primary context has been destroyed), when the library's
+ *   device image, and the array with it, may be loaded at another address.
  *   Every call shares the one array per device: calls that may run at the
  *   same time on the GPU (different streams, or different host threads)
  *   race and corrupt each other's results.  Nothing in the array has to start
@@ -205,7 +208,8 @@ LMH_API lmh_status_t ce_bwd_shard(const float *logits, const int64_t *target, co
                                   lmh_stream_t stream);
 
 /* dX = dlogits . W, the input gradient of logits = X . W^T
- * ([P1] "What does this PR do?", backward under the GEMM contract).
+ * ([P1] "What does this PR do?", backward under the GEMM contract: the
+ * gradient GEMMs take the BF16 dlogits cast from the FP32 backward).
  *   dlogits [M,V] BF16.  W [V,K] BF16.
  *   dX      [M,K] FP32 (LMH_F32) or BF16 (LMH_BF16).
  *   Requirements: V % 8 == 0 and K % 8 == 0 (16-byte rows), inputs 16-byte
@@ -214,7 +218,9 @@ LMH_API lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX,
                            int64_t M, int64_t K, int64_t V, int32_t *status,
                            lmh_stream_t stream);
 
-/* dW = dlogits^T . X, the weight gradient of logits = X . W^T.
+/* dW = dlogits^T . X, the weight gradient of logits = X . W^T
+ * ([P1] "What does this PR do?", backward under the GEMM contract: the
+ * gradient GEMMs take the BF16 dlogits cast from the FP32 backward).
  *   dlogits [M,V] BF16.  X [M,K] BF16.
  *   dW      [V,K] FP32 (LMH_F32) or BF16 (LMH_BF16).
  *   Requirements: V % 8 == 0 and K % 8 == 0, inputs 16-byte aligned.
@@ -249,6 +255,19 @@ LMH_API int32_t lmh_version(void);
  * (device int32, required).  Nothing faults or hangs; the context stays
  * usable.  Asynchronous like every other call. */
 LMH_API lmh_status_t lmh_watchdog_selftest(int32_t *status, int64_t limit_us, lmh_stream_t stream);
+
+/* Self-test of the GEMM's own failure path (failure detection; no
+ * counterpart on the pages).  Runs lmhead_fwd with FP32 logits, the same
+ * kernel selection and arguments, but with every pipeline wait limited to
+ * `limit_ns` nanoseconds (1..1000000000) instead of two seconds.  With a limit
+ * far below the time one output tile takes (1 ns, say), a wait runs out: the
+ * CTA stops, lets every operand copy it issued land and every MMA it issued
+ * finish, frees its tensor memory and ORs LMH_DEV_PIPE_TIMEOUT into *status
+ * (device int32, required).  The logits are then not valid.  Nothing faults
+ * or hangs, and later calls on the stream run normally. */
+LMH_API lmh_status_t lmh_gemm_watchdog_selftest(const void *X, const void *W, float *logits,
+                                                int64_t M, int64_t K, int64_t V, int64_t limit_ns,
+                                                int32_t *status, lmh_stream_t stream);
 
 #ifdef __cplusplus
 }

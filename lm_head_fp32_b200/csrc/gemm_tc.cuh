@@ -32,7 +32,10 @@
 // halve the epilogue of a tile, which matters where no MMA hides it: the last
 // tile of each CTA when the fused cross-entropy statistics lengthen it.
 // Every wait is bounded (see mbar_wait); on a timeout the CTA drains its own
-// copies and MMAs, frees tensor memory, sets a status bit and returns.
+// copies and MMAs, frees tensor memory, sets a status bit and returns.  A CTA
+// pair first settles, through distributed shared memory, which operand copies
+// either CTA has issued, completes the set, and waits for all of them to land
+// before either CTA leaves (see the end of the kernel).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -58,7 +61,17 @@ struct GemmParams {
     int32_t m_fastest;  // tile order: 1 = consecutive tiles share n (B panel)
     int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
     int32_t l2_b;
+    int32_t l2_out;     // L2 policy of the output stores (TMA store epilogue): 0 none, 1 evict first
     int32_t *status;
+    uint64_t wait_limit_ns;  // limit of every pipeline wait (the host sets kWaitLimitNs)
+    // The last split_tiles tiles of the tile order are each computed as two
+    // work items, the first and the second half of the k-blocks, whose FP32
+    // sums are both added (TMA reduce-add) into output the host has zeroed:
+    // fl(0 + a) = a and fl(a + b) = fl(b + a), so the result does not depend on
+    // which half lands first.  Used for a last wave that would leave most
+    // SMs idle; 0 = no split (requires two or more k-blocks).
+    int32_t split_tiles;
+    int32_t allow_split;  // host side: the call may split its last wave (FP32 output)
     // fused cross-entropy statistics (vocabulary GEMM only): per 128-wide
     // vocabulary block s (one CTA's rows of a tile) and token i,
     // ce_partial[s * Ndim + i] = (max, sum-exp) of the block (a warp stores
@@ -241,6 +254,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
     uint64_t *drain = bars + 2 * S + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile uint32_t *issued_sh = tmem_slot + 2;  // k-blocks whose copies this CTA issued
     // CE exchange: xch_full[2], xch_free[2], then xch[2][3][32] pairs
     uint64_t *xch_full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(bars) +
                                                       C::BAR_BYTES + 16);
@@ -255,6 +269,22 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
     const int num_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int num_tiles = p.num_m_tiles * p.num_n_tiles;
     const int num_kb = (p.Kdim + kBlockK - 1) / kBlockK;
+    const int split_first = num_tiles - p.split_tiles;
+    const int num_items = split_first + 2 * p.split_tiles;
+    // work item -> tile and k-block range [kb0, kb1); true for a half tile
+    auto item_of = [&](int it, int &t, int &kb0, int &kb1) -> bool {
+        if (it < split_first) {
+            t = it;
+            kb0 = 0;
+            kb1 = num_kb;
+            return false;
+        }
+        const int j = it - split_first;
+        t = split_first + (j >> 1);
+        kb0 = (j & 1) ? num_kb / 2 : 0;
+        kb1 = (j & 1) ? num_kb : num_kb / 2;
+        return true;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -273,6 +303,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
             }
         }
         *abort_flag = 0;
+        *issued_sh = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -297,59 +328,65 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
     pdl_wait();
     pdl_launch_dependents();
 
+    // Copies of one k-block into ring slot `stage`: this CTA's A rows from m0
+    // and B rows from nb0 at reduction offset k0.  The full barrier (the
+    // leader's, for a pair) counts the bytes of both CTAs; the leader arms it.
+    const uint64_t pol_a = policy_of(p.l2_a);
+    const uint64_t pol_b = policy_of(p.l2_b);
+    auto issue_kblock = [&](uint32_t stage, int m0, int nb0, int k0) {
+        uint8_t *sa = tiles + stage * C::STAGE_BYTES;
+        uint8_t *sb = sa + C::A_BYTES;
+        const uint32_t fb = PAIR ? mapa_shared(smem_u32(&full[stage]), 0) : 0u;
+        if (leader)
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES * C::CTAS);
+        if (A_MN) {
+#pragma unroll
+            for (int j = 0; j < kBlockM / 64; ++j) {
+                if (PAIR)
+                    tma_load_2d_pair(&tmA, fb, sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
+                else
+                    tma_load_2d(&tmA, &full[stage], sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
+            }
+        } else {
+            if (PAIR)
+                tma_load_2d_pair(&tmA, fb, sa, k0, m0, pol_a);
+            else
+                tma_load_2d(&tmA, &full[stage], sa, k0, m0, pol_a);
+        }
+        if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < C::BN_CTA / 64; ++j) {
+                if (PAIR)
+                    tma_load_2d_pair(&tmB, fb, sb + j * 64 * kBlockK * 2, nb0 + 64 * j, k0, pol_b);
+                else
+                    tma_load_2d(&tmB, &full[stage], sb + j * 64 * kBlockK * 2, nb0 + 64 * j, k0, pol_b);
+            }
+        } else {
+            if (PAIR)
+                tma_load_2d_pair(&tmB, fb, sb, k0, nb0, pol_b);
+            else
+                tma_load_2d(&tmB, &full[stage], sb, k0, nb0, pol_b);
+        }
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint64_t pol_a = policy_of(p.l2_a);
-            const uint64_t pol_b = policy_of(p.l2_b);
             uint32_t stage = 0, phase = 0;
-            int64_t issued = 0;
+            uint32_t issued = 0;
             bool ok = true;
-            for (int t = unit; t < num_tiles && ok; t += num_units) {
-                int mt, nt;
+            for (int it = unit; it < num_items && ok; it += num_units) {
+                int t, kb0, kb1, mt, nt;
+                item_of(it, t, kb0, kb1);
                 tile_coords(t, p, mt, nt);
                 const int m0 = mt * C::TILE_M + static_cast<int>(rank) * kBlockM;  // this CTA's A rows
                 const int nb0 = nt * BN + static_cast<int>(rank) * C::BN_CTA;     // this CTA's B rows
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
-                    uint8_t *sa = tiles + stage * C::STAGE_BYTES;
-                    uint8_t *sb = sa + C::A_BYTES;
-                    // the leader's full barrier counts the bytes of both CTAs
-                    const uint32_t fb = PAIR ? mapa_shared(smem_u32(&full[stage]), 0) : 0u;
-                    if (leader)
-                        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES * C::CTAS);
-                    const int k0 = kb * kBlockK;
-                    if (A_MN) {
-#pragma unroll
-                        for (int j = 0; j < kBlockM / 64; ++j) {
-                            if (PAIR)
-                                tma_load_2d_pair(&tmA, fb, sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
-                            else
-                                tma_load_2d(&tmA, &full[stage], sa + j * 64 * kBlockK * 2, m0 + 64 * j, k0, pol_a);
-                        }
-                    } else {
-                        if (PAIR)
-                            tma_load_2d_pair(&tmA, fb, sa, k0, m0, pol_a);
-                        else
-                            tma_load_2d(&tmA, &full[stage], sa, k0, m0, pol_a);
-                    }
-                    if (B_MN) {
-#pragma unroll
-                        for (int j = 0; j < C::BN_CTA / 64; ++j) {
-                            if (PAIR)
-                                tma_load_2d_pair(&tmB, fb, sb + j * 64 * kBlockK * 2, nb0 + 64 * j, k0, pol_b);
-                            else
-                                tma_load_2d(&tmB, &full[stage], sb + j * 64 * kBlockK * 2, nb0 + 64 * j, k0, pol_b);
-                        }
-                    } else {
-                        if (PAIR)
-                            tma_load_2d_pair(&tmB, fb, sb, k0, nb0, pol_b);
-                        else
-                            tma_load_2d(&tmB, &full[stage], sb, k0, nb0, pol_b);
-                    }
+                    issue_kblock(stage, m0, nb0, kb * kBlockK);
                     ++issued;
                     if (++stage == S) {
                         stage = 0;
@@ -357,17 +394,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                     }
                 }
             }
-            if (!ok) {
-                // let the copies already issued land before the CTA exits
-                if (PAIR) {
-                    sleep_ns(20000);  // the pair's barrier lives in the leader
-                } else {
-                    volatile int no_abort = 0;
-                    for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i)
-                        mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1), &no_abort,
-                                  kDrainLimitNs);
-                }
-            }
+            *issued_sh = issued;
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (pair: leader only)
@@ -375,15 +402,17 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
             uint32_t stage = 0, phase = 0;
             uint32_t acc = 0, acc_phase = 0;
             bool ok = true;
-            for (int t = unit; t < num_tiles && ok; t += num_units) {
-                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) {
+            for (int it = unit; it < num_items && ok; it += num_units) {
+                int t, kb0, kb1;
+                item_of(it, t, kb0, kb1);
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -398,10 +427,11 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                                                  : smem_desc_sw128(sa + k * 32, 16, 1024);
                         const uint64_t db = B_MN ? smem_desc_sw128(sb + k * 2048, 64 * kBlockK * 2, 1024)
                                                  : smem_desc_sw128(sb + k * 32, 16, 1024);
+                        const uint32_t accumulate = (kb != kb0 || k != 0) ? 1u : 0u;
                         if (PAIR)
-                            mma_bf16_pair(d_tmem, da, db, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                            mma_bf16_pair(d_tmem, da, db, C::IDESC, accumulate);
                         else
-                            mma_bf16(d_tmem, da, db, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                            mma_bf16(d_tmem, da, db, C::IDESC, accumulate);
                     }
                     // frees the smem slot (of both CTAs) when these MMAs finish
                     if (PAIR)
@@ -439,6 +469,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
         const int half = (warp - 2) >> 2;  // EW = 8: which alternate sub-tiles of the quarter
         const int row = q * 32 + lane;
         OutT *out = static_cast<OutT *>(p.out);
+        const uint64_t pol_out = policy_of(p.l2_out);
         OutT *slots = reinterpret_cast<OutT *>(epi_smem + (warp - 2) * C::NSLOT * C::EPI_SLOT_BYTES);
         constexpr int SLOT_ELEMS = C::EPI_SLOT_BYTES / static_cast<int>(sizeof(float));
         uint32_t slot = 0;
@@ -446,14 +477,15 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
         // where this warp releases an accumulator: the leader's barrier
         const uint32_t empty_addr0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
         uint32_t acc = 0, acc_phase = 0;
-        for (int t = unit; t < num_tiles; t += num_units) {
+        for (int it = unit; it < num_items; it += num_units) {
             // every lane waits, then the warp agrees, so the .sync.aligned
             // tensor-memory loads below always run with the full warp
-            const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
+            const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok))
                 break;
             tc_fence_after();
-            int mt, nt;
+            int t, kb0, kb1, mt, nt;
+            const bool half_tile = item_of(it, t, kb0, kb1);
             tile_coords(t, p, mt, nt);
             const int mbase = mt * C::TILE_M + static_cast<int>(rank) * kBlockM;
             const int m = mbase + row;
@@ -480,8 +512,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        if (ACC)
+                        if (ACC || half_tile)
                             tma_reduce_add_2d(&tmC, buf, mbase + q * 32, n0 + c);
+                        else if (p.l2_out)
+                            tma_store_2d_hint(&tmC, buf, mbase + q * 32, n0 + c, pol_out);
                         else
                             tma_store_2d(&tmC, buf, mbase + q * 32, n0 + c);
                         bulk_commit();
@@ -501,13 +535,14 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                                              C::EPI_CHUNK, mbase + q * 32, p.Mdim, tok, p.Ndim, p);
                         MaxSum *xh = xch + half * 3 * 32;
                         if (q != 0) {
-                            if (mbar_wait(&xch_free[half], xch_phase ^ 1, abort_flag))
+                            if (mbar_wait(&xch_free[half], xch_phase ^ 1, abort_flag, p.wait_limit_ns))
                                 xh[(q - 1) * 32 + lane] = sv;
                             __syncwarp();
                             if (lane == 0)
                                 mbar_arrive(&xch_full[half]);
                         } else {
-                            const bool got = mbar_wait(&xch_full[half], xch_phase, abort_flag);
+                            const bool got =
+                                mbar_wait(&xch_full[half], xch_phase, abort_flag, p.wait_limit_ns);
                             MaxSum r = sv;
                             if (got) {
 #pragma unroll
@@ -530,7 +565,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
 #pragma unroll
                     for (int j = 0; j < C::EPI_CHUNK; ++j)
                         if (n0 + c + j < p.Ndim) {
-                            if constexpr (ACC)
+                            // FP32 only: an accumulating or half-tile store adds
+                            if (sizeof(OutT) == 4 && (ACC || half_tile))
                                 atomicAdd(reinterpret_cast<float *>(o) + static_cast<int64_t>(j) * p.ldo,
                                           __uint_as_float(r[j]));
                             else
@@ -557,10 +593,51 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
 
     tc_fence_before();
     __syncthreads();
-    if (PAIR) {
-        if (*abort_flag)
-            sleep_ns(20000);  // copies or arrivals of the peer still in flight
-        cluster_sync();       // both CTAs are done with tensor memory and barriers
+    if constexpr (PAIR) {
+        // Every role of both CTAs has finished (the leader's MMAs are
+        // drained); the abort flags and issued counts are final.
+        cluster_sync();
+        const uint32_t peer = rank ^ 1u;
+        const int peer_abort = static_cast<int>(
+            ld_shared_cluster_u32(mapa_shared(smem_u32(const_cast<int *>(abort_flag)), peer)));
+        if (*abort_flag || peer_abort) {
+            // After a timeout the two producers may have stopped at different
+            // k-blocks, so the leader's full barriers may wait for bytes that
+            // will never come, or copies may still be landing in either CTA.
+            // A k-block issued by one CTA implies that the MMAs of the
+            // k-block S earlier in its slot completed, hence that slot's
+            // previous phase completed in both CTAs.  So the CTA that is
+            // behind can issue (and the leader arm) the k-blocks it missed;
+            // every issued copy then belongs to a phase that completes, and
+            // the leader waits for the last phase of each slot.  The copied
+            // data is not used.
+            if (threadIdx.x == 0) {
+                const uint32_t mine = *issued_sh;
+                const uint32_t theirs = ld_shared_cluster_u32(
+                    mapa_shared(smem_u32(const_cast<uint32_t *>(issued_sh)), peer));
+                const uint32_t all = mine > theirs ? mine : theirs;
+                for (uint32_t i = mine; i < all; ++i)
+                    issue_kblock(i % S, static_cast<int>(rank) * kBlockM,
+                                 static_cast<int>(rank) * C::BN_CTA, 0);
+                if (leader) {
+                    volatile int no_abort = 0;
+                    for (uint32_t i = all > S ? all - S : 0; i < all; ++i)
+                        mbar_wait(&full[i % S], (i / S) & 1u, &no_abort, kDrainLimitNs);
+                }
+            }
+            cluster_sync();  // every copy into either CTA has landed
+        }
+        cluster_sync();  // neither CTA reads the other's shared memory any more
+    } else {
+        if (*abort_flag && threadIdx.x == 0) {
+            // Copies issued but never consumed may still be landing: wait for
+            // the last phase of each slot (older phases completed before
+            // their slots were refilled).  The CTA stays resident meanwhile.
+            const uint32_t all = *issued_sh;
+            volatile int no_abort = 0;
+            for (uint32_t i = all > S ? all - S : 0; i < all; ++i)
+                mbar_wait(&full[i % S], (i / S) & 1u, &no_abort, kDrainLimitNs);
+        }
     }
     if (warp == 1) {
         __syncwarp();

@@ -7,7 +7,6 @@
 
 #include <atomic>
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -107,15 +106,16 @@ lmh_status_t last_cuda_error()
     return cudaGetLastError() == cudaSuccess ? LMH_OK : LMH_ERR_CUDA;
 }
 
-// Programmatic dependent launch is on unless LMH_PDL=0 is set in the
-// environment (a tuning aid; read once per process).
-bool pdl_enabled()
+// Programmatic dependent launch is on unless the library is built with
+// -DLMH_NO_PDL (a build-time switch for measurements; nothing in the
+// environment changes the kernels a call launches).
+constexpr bool pdl_enabled()
 {
-    static const bool on = [] {
-        const char *e = std::getenv("LMH_PDL");
-        return !(e && e[0] == '0');
-    }();
-    return on;
+#ifdef LMH_NO_PDL
+    return false;
+#else
+    return true;
+#endif
 }
 
 // Launch with programmatic stream serialisation allowed (the kernel waits in
@@ -191,6 +191,8 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
             return LMH_ERR_CUDA;
         attr_set.fetch_or(bit);
     }
+    if (p.wait_limit_ns == 0)
+        p.wait_limit_ns = lmh::kWaitLimitNs;
     p.num_m_tiles = static_cast<int32_t>((p.Mdim + C::TILE_M - 1) / C::TILE_M);
     p.num_n_tiles = static_cast<int32_t>((p.Ndim + BN - 1) / BN);
     const int64_t tiles = static_cast<int64_t>(p.num_m_tiles) * p.num_n_tiles;
@@ -198,7 +200,27 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
         return LMH_ERR_INVALID_ARG;
     // persistent: one CTA (or CTA pair) per SM (pair); several resident per SM: one per tile
     const int64_t units = RES == 1 ? num_sms() / C::CTAS : tiles;
-    const int grid = static_cast<int>((tiles < units ? tiles : units) * C::CTAS);
+    p.split_tiles = 0;
+    if constexpr (TMA_STORE && sizeof(OutT) == 4 && !CE && !ACC && RES == 1) {
+        // A last wave of rem tiles on `units` SMs (pairs) that would leave
+        // more than half of them idle: split those tiles into two k-halves
+        // that both add into zeroed output (deterministic: two addends).
+        // With tiles in m-fastest order they are the last n-rows of the
+        // output, which are contiguous, so one memset zeroes them.
+        const int64_t rem = tiles % units;
+        const int64_t num_kb = (p.Kdim + lmh::kBlockK - 1) / lmh::kBlockK;
+        if (p.allow_split && p.m_fastest && tiles > units && rem > 0 && 2 * rem <= units &&
+            num_kb >= 2) {
+            p.split_tiles = static_cast<int32_t>(rem);
+            const int64_t row0 = ((tiles - rem) / p.num_m_tiles) * BN;
+            const size_t bytes = static_cast<size_t>(p.Ndim - row0) * p.ldo * sizeof(float);
+            if (cudaMemsetAsync(static_cast<float *>(p.out) + row0 * p.ldo, 0, bytes, stream) !=
+                cudaSuccess)
+                return LMH_ERR_CUDA;
+        }
+    }
+    const int64_t items = tiles + p.split_tiles;
+    const int grid = static_cast<int>((items < units ? items : units) * C::CTAS);
     return launch_ex(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream,
                      PAIR ? 2u : 1u, ta, tb, tc, p);
 }
@@ -245,23 +267,30 @@ int pick_bn_tokens(int64_t M)
     return 256;
 }
 
+// L2 policy of the logits the vocabulary GEMM stores.  Evict first: while the
+// tensor-bound GEMM still streams W through L2, its logit lines are the first
+// to be written back, so the kernel that reads them next does not inherit a
+// cache full of dirty lines to write back under its own reads.
+#ifndef LMH_LOGITS_L2_POLICY
+#define LMH_LOGITS_L2_POLICY 1
+#endif
+constexpr int kLogitsL2Policy = LMH_LOGITS_L2_POLICY;
+
 // L2 policy of W in the vocabulary GEMM: streamed once (evict first) when a
 // single token tile reads each W panel, normal when several token tiles reuse
 // it (measured: +13 % for M <= 128, -7 % at M = 1024 with evict first).
 int w_policy(int64_t M, int bn) { return M <= bn ? 1 : 0; }
 
 // CTA-pair tiles (256 x 256) are used when the n extent fills a 256-wide
-// tile.  LMH_GEMM_PAIR=0 or 1 in the environment forces single-CTA or pair
-// tiles where both are possible (a tuning aid; read once per process).
-int pair_override()
+// tile.  Building with -DLMH_GEMM_PAIR=0 or =1 forces single-CTA or pair tiles
+// where both are possible (a build-time switch for measurements).
+constexpr int pair_override()
 {
-    static int v = [] {
-        const char *e = std::getenv("LMH_GEMM_PAIR");
-        if (!e || !*e)
-            return -1;
-        return e[0] == '0' ? 0 : 1;
-    }();
-    return v;
+#ifdef LMH_GEMM_PAIR
+    return LMH_GEMM_PAIR ? 1 : 0;
+#else
+    return -1;
+#endif
 }
 
 bool use_pair(int bn, int64_t Mdim)
@@ -384,6 +413,38 @@ bool dims_ok(int64_t a, int64_t b, int64_t c)
     return a >= 1 && b >= 1 && c >= 1 && a <= kMaxDim && b <= kMaxDim && c <= kMaxDim;
 }
 
+// lmhead_fwd with a given pipeline wait limit (0: the default limit).
+lmh_status_t fwd_impl(const void *X, const void *W, void *logits, int32_t out_dtype, int64_t M,
+                      int64_t K, int64_t V, int32_t *status, lmh_stream_t stream,
+                      uint64_t wait_limit_ns)
+{
+    if (!X || !W || !logits || !dims_ok(M, K, V))
+        return LMH_ERR_INVALID_ARG;
+    if (bad_dtype(out_dtype))
+        return LMH_ERR_UNSUPPORTED;
+    if (K % 8 || !aligned(X, 16) || !aligned(W, 16) ||
+        !aligned(logits, out_dtype == LMH_F32 ? 4 : 2))
+        return LMH_ERR_MISALIGNED;
+    const int bn = pick_bn_tokens(M);
+    const Operand a{W, static_cast<uint64_t>(K), static_cast<uint64_t>(V), false};  // A = W
+    const Operand b{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), false};  // B = X
+    GemmParams p{};
+    p.out = logits;
+    p.ldo = V;
+    p.Mdim = static_cast<int32_t>(V);
+    p.Ndim = static_cast<int32_t>(M);
+    p.Kdim = static_cast<int32_t>(K);
+    p.m_fastest = 0;  // consecutive tiles share one W panel
+    p.l2_a = w_policy(M, bn);
+    p.l2_b = 2;  // X is reread by every tile
+    p.l2_out = kLogitsL2Policy;
+    p.status = status;
+    p.wait_limit_ns = wait_limit_ns;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, a, b, p, s)
+                                : dispatch_bn<false, false, __nv_bfloat16>(bn, a, b, p, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -414,29 +475,17 @@ lmh_status_t lmh_watchdog_selftest(int32_t *status, int64_t limit_us, lmh_stream
 lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int32_t out_dtype, int64_t M,
                         int64_t K, int64_t V, int32_t *status, lmh_stream_t stream)
 {
-    if (!X || !W || !logits || !dims_ok(M, K, V))
+    return fwd_impl(X, W, logits, out_dtype, M, K, V, status, stream, 0);
+}
+
+lmh_status_t lmh_gemm_watchdog_selftest(const void *X, const void *W, float *logits, int64_t M,
+                                        int64_t K, int64_t V, int64_t limit_ns, int32_t *status,
+                                        lmh_stream_t stream)
+{
+    if (!status || limit_ns < 1 || limit_ns > 1000000000)
         return LMH_ERR_INVALID_ARG;
-    if (bad_dtype(out_dtype))
-        return LMH_ERR_UNSUPPORTED;
-    if (K % 8 || !aligned(X, 16) || !aligned(W, 16) ||
-        !aligned(logits, out_dtype == LMH_F32 ? 4 : 2))
-        return LMH_ERR_MISALIGNED;
-    const int bn = pick_bn_tokens(M);
-    const Operand a{W, static_cast<uint64_t>(K), static_cast<uint64_t>(V), false};  // A = W
-    const Operand b{X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), false};  // B = X
-    GemmParams p{};
-    p.out = logits;
-    p.ldo = V;
-    p.Mdim = static_cast<int32_t>(V);
-    p.Ndim = static_cast<int32_t>(M);
-    p.Kdim = static_cast<int32_t>(K);
-    p.m_fastest = 0;  // consecutive tiles share one W panel
-    p.l2_a = w_policy(M, bn);
-    p.l2_b = 2;  // X is reread by every tile
-    p.status = status;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return out_dtype == LMH_F32 ? dispatch_bn<false, false, float>(bn, a, b, p, s)
-                                : dispatch_bn<false, false, __nv_bfloat16>(bn, a, b, p, s);
+    return fwd_impl(X, W, logits, LMH_F32, M, K, V, status, stream,
+                    static_cast<uint64_t>(limit_ns));
 }
 
 lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t out_dtype,
@@ -463,6 +512,7 @@ lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t
     p.l2_a = 0;  // every W and dlogits chunk is read by the concurrently running tiles
     p.l2_b = 0;
     p.status = status;
+    p.allow_split = 1;  // few output tiles, each with a long reduction over V
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return out_dtype == LMH_F32 ? dispatch_bn<true, false, float>(bn, a, b, p, s)
                                 : dispatch_bn<true, false, __nv_bfloat16>(bn, a, b, p, s);
@@ -566,6 +616,7 @@ lmh_status_t lmhead_fwd_ce(const void *X, const void *W, const int64_t *target, 
     p.m_fastest = 0;
     p.l2_a = w_policy(M, bn);
     p.l2_b = 2;
+    p.l2_out = kLogitsL2Policy;
     p.status = status;
     p.ce_partial = static_cast<float2 *>(workspace);
     p.ce_target = target;
@@ -782,6 +833,7 @@ extern "C" lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, cons
     p.m_fastest = 0;
     p.l2_a = w_policy(M, bn);
     p.l2_b = 2;
+    p.l2_out = kLogitsL2Policy;
     p.status = status;
     p.ce_partial = scratch;
     p.ce_target = target;

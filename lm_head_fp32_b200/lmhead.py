@@ -25,7 +25,8 @@ IGNORE_INDEX = -100
 EXPORTS = ("lmhead_fwd", "ce_fwd", "ce_bwd", "lmhead_bwd_dx", "lmhead_bwd_dw",
            "lmhead_fwd_ce", "lmhead_fwd_ce_workspace_bytes", "lmhead_fwd_ce_noalloc",
            "lmhead_bwd_dw_acc", "ce_fwd_shard", "ce_merge_shards", "ce_bwd_shard",
-           "lmh_status_string", "lmh_version", "lmh_watchdog_selftest")
+           "lmh_status_string", "lmh_version", "lmh_watchdog_selftest",
+           "lmh_gemm_watchdog_selftest")
 
 _lib = None
 
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.lmhead_fwd_ce_workspace_bytes.restype = I64
         L.lmh_watchdog_selftest.argtypes = [P, I64, P]
         L.lmh_watchdog_selftest.restype = ctypes.c_int
+        L.lmh_gemm_watchdog_selftest.argtypes = [P, P, P, I64, I64, I64, I64, P, P]
+        L.lmh_gemm_watchdog_selftest.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -220,6 +223,19 @@ def watchdog_selftest(status: torch.Tensor, limit_us: int = 1000, stream=None) -
     """Make one bounded pipeline wait run out on purpose; sets DEV_PIPE_TIMEOUT."""
     _check(lib().lmh_watchdog_selftest(_ptr(status), int(limit_us), _stream(stream)),
            "lmh_watchdog_selftest")
+
+
+def gemm_watchdog_selftest(X: torch.Tensor, W: torch.Tensor, logits: torch.Tensor,
+                           status: torch.Tensor, limit_ns: int = 1, stream=None) -> None:
+    """lmhead_fwd (FP32 logits) with every pipeline wait limited to limit_ns:
+    the GEMM's own timeout path, which sets DEV_PIPE_TIMEOUT."""
+    _contig(X, W, logits)
+    M, K = X.shape
+    V = W.shape[0]
+    assert W.shape[1] == K and tuple(logits.shape) == (M, V) and logits.dtype == torch.float32
+    _check(lib().lmh_gemm_watchdog_selftest(_ptr(X), _ptr(W), _ptr(logits), M, K, V,
+                                            int(limit_ns), _ptr(status), _stream(stream)),
+           "lmh_gemm_watchdog_selftest")
 
 
 def lmhead_bwd_dw_acc(dlogits: torch.Tensor, X: torch.Tensor, dW: torch.Tensor,

@@ -19,7 +19,7 @@ binding and exists so that the sequencing can be exercised without a GPU.
 """
 from __future__ import annotations
 
-from typing import Optional
+from typing import Callable, Optional
 
 import torch
 import torch.distributed as dist
@@ -29,46 +29,79 @@ from . import lmhead as _lmhead
 
 def shard_bounds(vocab_total: int, world: int, rank: int, multiple: int = 8):
     """[offset, offset + size) of rank's shard: near-equal sizes, each a
-    multiple of `multiple` entries except possibly the last."""
+    multiple of `multiple` entries except possibly the last.  When the
+    vocabulary is small for the world size the last ranks' shards are empty
+    (size 0); step() handles those."""
     per = -(-vocab_total // world)
     per = -(-per // multiple) * multiple
     off = min(rank * per, vocab_total)
     return off, min(per, vocab_total - off)
 
 
+STAGES = ("lmhead_fwd", "ce_fwd_shard", "all_gather", "ce_merge_shards", "ce_bwd_shard",
+          "lmhead_bwd_dx", "all_reduce", "lmhead_bwd_dw")
+
+
 def step(X: torch.Tensor, W_shard: torch.Tensor, target: torch.Tensor, vocab_offset: int,
          vocab_total: int, grad_loss: torch.Tensor, group=None, ignore_index: int = -100,
-         status: Optional[torch.Tensor] = None, ops=None):
+         status: Optional[torch.Tensor] = None, ops=None,
+         mark: Optional[Callable[[str], None]] = None):
     """One vocabulary-parallel forward + backward on this rank.
+
+    `mark`, if given, is called with each name of STAGES, in that order, right
+    after that stage has been enqueued (a timing hook).
 
     Returns (stats[M,4] of the whole vocabulary, dX[M,K] summed over ranks,
     dW_shard[V_r,K], logits_shard, dl_shard)."""
     ops = ops or _lmhead
+    mark = mark or (lambda name: None)
     M, K = X.shape
     Vr = W_shard.shape[0]
     dev = X.device
     world = dist.get_world_size(group) if dist.is_initialized() else 1
 
     logits = torch.empty((M, Vr), dtype=torch.float32, device=dev)
-    ops.lmhead_fwd(X, W_shard, logits, status)
     rec = torch.empty((M, 4), dtype=torch.float32, device=dev)
-    ops.ce_fwd_shard(logits, target, rec, vocab_offset, vocab_total, ignore_index, status)
+    if Vr > 0:
+        ops.lmhead_fwd(X, W_shard, logits, status)
+        mark("lmhead_fwd")
+        ops.ce_fwd_shard(logits, target, rec, vocab_offset, vocab_total, ignore_index, status)
+        mark("ce_fwd_shard")
+    else:
+        # an empty shard contributes the neutral record (no maximum, no mass,
+        # no target) and no gradient, but still joins both collectives, so
+        # that every rank takes the same steps
+        rec.zero_()
+        rec[:, 0] = float("-inf")
+        mark("lmhead_fwd")
+        mark("ce_fwd_shard")
     if world > 1:
-        parts = [torch.empty_like(rec) for _ in range(world)]
-        dist.all_gather(parts, rec, group=group)
-        recs = torch.stack(parts)
+        recs = torch.empty((world * M, 4), dtype=torch.float32, device=dev)
+        dist.all_gather_into_tensor(recs, rec, group=group)
+        recs = recs.view(world, M, 4)
     else:
         recs = rec.unsqueeze(0)
+    mark("all_gather")
     stats = torch.empty((M, 4), dtype=torch.float32, device=dev)
-    ops.ce_merge_shards(recs.contiguous(), target, stats, vocab_total, ignore_index, status)
+    ops.ce_merge_shards(recs, target, stats, vocab_total, ignore_index, status)
+    mark("ce_merge_shards")
 
     dl = torch.empty((M, Vr), dtype=torch.bfloat16, device=dev)
-    ops.ce_bwd_shard(logits, target, stats, grad_loss, dl, vocab_offset, vocab_total,
-                     ignore_index, status)
     dX = torch.empty((M, K), dtype=torch.float32, device=dev)
-    ops.lmhead_bwd_dx(dl, W_shard, dX, status)
+    if Vr > 0:
+        ops.ce_bwd_shard(logits, target, stats, grad_loss, dl, vocab_offset, vocab_total,
+                         ignore_index, status)
+        mark("ce_bwd_shard")
+        ops.lmhead_bwd_dx(dl, W_shard, dX, status)
+    else:
+        mark("ce_bwd_shard")
+        dX.zero_()
+    mark("lmhead_bwd_dx")
     if world > 1:
         dist.all_reduce(dX, op=dist.ReduceOp.SUM, group=group)
+    mark("all_reduce")
     dW = torch.empty((Vr, K), dtype=torch.float32, device=dev)
-    ops.lmhead_bwd_dw(dl, X, dW, status)
+    if Vr > 0:
+        ops.lmhead_bwd_dw(dl, X, dW, status)
+    mark("lmhead_bwd_dw")
     return stats, dX, dW, logits, dl

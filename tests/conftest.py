@@ -16,3 +16,13 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(autouse=True)
+def _guard_bands(request):
+    """After every GPU test: the guard bands around each output made with
+    helpers.guarded_empty are untouched."""
+    yield
+    if request.node.get_closest_marker("gpu") is not None:
+        import helpers
+        helpers.check_guards()

@@ -13,6 +13,13 @@ Tolerances, from the contract the tests enforce:
     cancellation that exceeds one BF16 ulp of the tiny result, so for GEMM
     outputs the bound is one ulp plus the FP32 tolerance (abs_tol);
   * dX / dW on random inputs: 1e-5 * sqrt(reduction length) * max|a| * max|b|.
+
+Out-of-bounds writes: every GPU output of the parity tests comes from
+guarded_empty(), which places it between two 4 KiB guard bands filled with
+0xFF bytes (a NaN in FP32 and in BF16, a value no kernel here writes); after
+each GPU test the bands of every such buffer are checked (tests/conftest.py),
+so a ragged tile or a partial vocabulary block that writes past its output is
+caught even where the output's own values look right.
 """
 from __future__ import annotations
 
@@ -22,6 +29,49 @@ import numpy as np
 import torch
 
 import oracle
+
+
+GUARD_BYTES = 4096
+GUARD_FILL = 0xFF
+_guarded = []
+
+
+def guarded_empty(shape, dtype=torch.float32, device="cuda") -> torch.Tensor:
+    """A contiguous output tensor with GUARD_BYTES of GUARD_FILL bytes just
+    before and just after it (in the same allocation; the output stays
+    16-byte aligned).  Its own contents are GUARD_FILL bytes too."""
+    esize = torch.empty((), dtype=dtype).element_size()
+    nb = GUARD_BYTES // esize
+    n = math.prod(shape)
+    raw = torch.empty(n + 2 * nb, dtype=dtype, device=device)
+    raw.view(torch.uint8).fill_(GUARD_FILL)
+    _guarded.append((raw, nb, n))
+    return raw[nb:nb + n].view(tuple(shape))
+
+
+def guarded_full(shape, value, dtype=torch.float32, device="cuda") -> torch.Tensor:
+    t = guarded_empty(shape, dtype, device)
+    t.fill_(value)
+    return t
+
+
+def check_guards():
+    """Assert that no guard band of a buffer made since the last check was
+    written, then forget those buffers."""
+    if not _guarded:
+        return
+    torch.cuda.synchronize()
+    bad = []
+    for raw, nb, n in _guarded:
+        b = raw.view(torch.uint8)
+        esize = raw.element_size()
+        for name, band in (("before", b[:nb * esize]), ("after", b[(nb + n) * esize:])):
+            hit = torch.nonzero(band != GUARD_FILL).flatten()
+            if hit.numel():
+                bad.append(f"{tuple(raw.shape)} {raw.dtype}: {hit.numel()} bytes written {name} "
+                           f"the output (first at band offset {int(hit[0])})")
+    _guarded.clear()
+    assert not bad, "; ".join(bad)
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
@@ -76,3 +126,59 @@ def gemm_tol(red_len: int, a: torch.Tensor, b: torch.Tensor) -> float:
 
 def loss_tol(ref: np.ndarray) -> np.ndarray:
     return 1e-5 * np.abs(ref) + 1e-6
+
+
+class FakeOps:
+    """float64 restatement of the library calls' contracts, on CPU tensors."""
+
+    @staticmethod
+    def lmhead_fwd(X, W, out, status=None):
+        out.copy_((X.double() @ W.double().T).float())
+
+    @staticmethod
+    def ce_fwd_shard(logits, target, rec, off, vtot, ignore, status=None):
+        x = logits.double().numpy()
+        V = x.shape[1]
+        r = np.zeros((x.shape[0], 4))
+        for i, y in enumerate(target.tolist()):
+            if y == ignore or y < 0 or y >= vtot:
+                continue
+            m = x[i].max()
+            own = off <= y < off + V
+            r[i] = (m, np.exp(x[i] - m).sum(), x[i, y - off] if own else 0.0, 1.0 if own else 0.0)
+        rec.copy_(torch.from_numpy(r).float())
+
+    @staticmethod
+    def ce_merge_shards(recs, target, stats, vtot, ignore, status=None):
+        R = recs.double().numpy()
+        out = np.zeros((R.shape[1], 4))
+        for i, y in enumerate(target.tolist()):
+            if y == ignore or y < 0 or y >= vtot:
+                continue
+            m = R[:, i, 0].max()
+            d = (R[:, i, 1] * np.exp(R[:, i, 0] - m)).sum()
+            xy = R[R[:, i, 3] != 0, i, 2].sum()
+            out[i] = (m, d, xy, m + np.log(d) - xy)
+        stats.copy_(torch.from_numpy(out).float())
+
+    @staticmethod
+    def ce_bwd_shard(logits, target, stats, g, dl, off, vtot, ignore, status=None):
+        x = logits.double().numpy()
+        st = stats.double().numpy()
+        out = np.zeros_like(x)
+        for i, y in enumerate(target.tolist()):
+            if y == ignore or y < 0 or y >= vtot:
+                continue
+            out[i] = np.exp(x[i] - st[i, 0]) / st[i, 1]
+            if off <= y < off + x.shape[1]:
+                out[i, y - off] -= 1.0
+            out[i] *= float(g.reshape(-1)[0])
+        dl.copy_(torch.from_numpy(out).to(dl.dtype))
+
+    @staticmethod
+    def lmhead_bwd_dx(dl, W, dX, status=None):
+        dX.copy_((dl.double() @ W.double()).float())
+
+    @staticmethod
+    def lmhead_bwd_dw(dl, X, dW, status=None):
+        dW.copy_((dl.double().T @ X.double()).float())

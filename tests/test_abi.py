@@ -109,6 +109,15 @@ def test_watchdog_selftest_validation():
     assert L.lmh_watchdog_selftest(A, 2000000, NULL) == lmhead.LMH_ERR_INVALID_ARG
 
 
+def test_gemm_watchdog_selftest_validation():
+    f = lmhead.lib().lmh_gemm_watchdog_selftest
+    assert f(A, A, A, 16, 64, 64, 1, NULL, NULL) == lmhead.LMH_ERR_INVALID_ARG   # no status
+    assert f(A, A, A, 16, 64, 64, 0, A, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert f(A, A, A, 16, 64, 64, 2000000000, A, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert f(NULL, A, A, 16, 64, 64, 1, A, NULL) == lmhead.LMH_ERR_INVALID_ARG
+    assert f(A, A, A, 16, 60, 64, 1, A, NULL) == lmhead.LMH_ERR_MISALIGNED       # K % 8
+
+
 def test_fused_ce_workspace_size_and_validation():
     L = lmhead.lib()
     # two 128-wide vocabulary blocks per 256 columns, one (max, sum-exp) pair each per token

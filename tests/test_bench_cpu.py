@@ -14,7 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_reference_arm_prints_one_complete_line():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
-                          "--warmup", "0", "--cpu-sample", "2"], cwd=ROOT, capture_output=True,
+                          "--warmup", "0", "--cpu-sample", "2", "--workload",
+                          "lmhead_1024x4096x32768"], cwd=ROOT, capture_output=True,
                          text=True, timeout=600, check=True)
     lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1
@@ -36,6 +37,20 @@ def test_reference_sample_shrinks_with_the_step_count():
     assert bench.reference_tokens_per_step(5, 1, 256) == 16
     assert bench.reference_tokens_per_step(5, 1, 2) == 2
     assert bench.reference_tokens_per_step(100000, 0, 256) == 1
+    # a token of the large-vocabulary workload costs ~3.9x one of the mid-size one
+    assert bench.reference_tokens_per_step(20, 5, 256, 4096, 128256) == 9
+
+
+def test_default_workload_is_the_large_vocabulary_lm_head(monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    args = bench.parse()
+    assert args.workload == "lmhead_4096x4096x128256"
+    cfg = bench.lmhead_config(args.workload)
+    assert (cfg.M, cfg.K, cfg.V, cfg.ignore_frac) == (4096, 4096, 128256, 0.01)
+    mid = bench.lmhead_config("lmhead_1024x4096x32768")
+    assert (mid.M, mid.ignore_frac) == (1024, 0.02)
+    other = bench.lmhead_config("lmhead_4096x4096x32768")
+    assert (other.M, other.K, other.V, other.dist) == (4096, 4096, 32768, "normal")
 
 
 def test_traffic_summary_is_tied_to_workload_and_sources():

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from lm_head_fp32_b200 import lmhead, synth
-from helpers import assert_abs_close, assert_bf16_close, loss_tol, to_f64
+from helpers import assert_abs_close, assert_bf16_close, guarded_empty, loss_tol, to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -18,11 +18,11 @@ DEV = "cuda"
 def run_ce(x: torch.Tensor, t: torch.Tensor, g, dl_dtype=torch.float32, ignore=-100):
     """x, t on the device; g: python float (stride 0) or a [M] FP32 tensor."""
     M, V = x.shape
-    st = torch.empty((M, 4), dtype=torch.float32, device=DEV)
+    st = guarded_empty((M, 4), torch.float32)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     lmhead.ce_fwd(x, t, st, ignore, status)
     gl = torch.tensor([g], dtype=torch.float32, device=DEV) if not torch.is_tensor(g) else g.to(DEV)
-    dl = torch.empty((M, V), dtype=dl_dtype, device=DEV)
+    dl = guarded_empty((M, V), dl_dtype)
     lmhead.ce_bwd(x, t, st, gl, dl, ignore, status)
     torch.cuda.synchronize()
     return st, dl, int(status.item())

@@ -17,7 +17,7 @@ import torch
 
 import oracle
 from lm_head_fp32_b200 import lmhead, synth
-from helpers import bits
+from helpers import bits, guarded_empty
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -39,8 +39,8 @@ def test_fp32_output_reduces_error_at_every_width():
         W = synth.normal_bf16((V, K), 0.02, 1235)
         t = synth.targets(M, V, 0.0, 1234).numpy()
         Xd, Wd = X.to(DEV), W.to(DEV)
-        l32 = torch.empty((M, V), dtype=torch.float32, device=DEV)
-        l16 = torch.empty((M, V), dtype=torch.bfloat16, device=DEV)
+        l32 = guarded_empty((M, V), torch.float32)
+        l16 = guarded_empty((M, V), torch.bfloat16)
         st = torch.zeros(1, dtype=torch.int32, device=DEV)
         lmhead.lmhead_fwd(Xd, Wd, l32, st)
         lmhead.lmhead_fwd(Xd, Wd, l16, st)

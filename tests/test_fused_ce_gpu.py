@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from lm_head_fp32_b200 import lmhead, synth
-from helpers import assert_abs_close, bits, logits_tol, loss_tol
+from helpers import assert_abs_close, bits, guarded_empty, logits_tol, loss_tol
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -15,9 +15,9 @@ DEV = "cuda"
 
 def fused(X, W, t, ignore=-100):
     M, V = X.shape[0], W.shape[0]
-    logits = torch.empty((M, V), dtype=torch.float32, device=DEV)
-    stats = torch.empty((M, 4), dtype=torch.float32, device=DEV)
-    ws = torch.empty(max(lmhead.lmhead_fwd_ce_workspace_bytes(M, V), 16), dtype=torch.uint8,
+    logits = guarded_empty((M, V), torch.float32)
+    stats = guarded_empty((M, 4), torch.float32)
+    ws = guarded_empty((max(lmhead.lmhead_fwd_ce_workspace_bytes(M, V), 16),), torch.uint8,
                      device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     lmhead.lmhead_fwd_ce(X.to(DEV), W.to(DEV), t.to(DEV), logits, stats, ws, ignore, status)
@@ -27,8 +27,8 @@ def fused(X, W, t, ignore=-100):
 
 def separate(X, W, t, ignore=-100):
     M, V = X.shape[0], W.shape[0]
-    logits = torch.empty((M, V), dtype=torch.float32, device=DEV)
-    stats = torch.empty((M, 4), dtype=torch.float32, device=DEV)
+    logits = guarded_empty((M, V), torch.float32)
+    stats = guarded_empty((M, 4), torch.float32)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     lmhead.lmhead_fwd(X.to(DEV), W.to(DEV), logits, status)
     lmhead.ce_fwd(logits, t.to(DEV), stats, ignore, status)

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from lm_head_fp32_b200 import lmhead, synth
-from helpers import assert_abs_close, assert_bf16_close, bits, gemm_tol, logits_tol, to_f64
+from helpers import assert_abs_close, assert_bf16_close, bits, gemm_tol, guarded_empty, guarded_full, logits_tol, to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -25,7 +25,7 @@ def status_word():
 
 def gpu_logits(X, W, dtype=torch.float32):
     M, V = X.shape[0], W.shape[0]
-    out = torch.empty((M, V), dtype=dtype, device=DEV)
+    out = guarded_empty((M, V), dtype)
     st = status_word()
     lmhead.lmhead_fwd(X.to(DEV), W.to(DEV), out, st)
     torch.cuda.synchronize()
@@ -34,7 +34,7 @@ def gpu_logits(X, W, dtype=torch.float32):
 
 
 def gpu_dx(dl, W, dtype=torch.float32):
-    out = torch.empty((dl.shape[0], W.shape[1]), dtype=dtype, device=DEV)
+    out = guarded_empty((dl.shape[0], W.shape[1]), dtype)
     st = status_word()
     lmhead.lmhead_bwd_dx(dl.to(DEV), W.to(DEV), out, st)
     torch.cuda.synchronize()
@@ -43,7 +43,7 @@ def gpu_dx(dl, W, dtype=torch.float32):
 
 
 def gpu_dw(dl, X, dtype=torch.float32):
-    out = torch.empty((dl.shape[1], X.shape[1]), dtype=dtype, device=DEV)
+    out = guarded_empty((dl.shape[1], X.shape[1]), dtype)
     st = status_word()
     lmhead.lmhead_bwd_dw(dl.to(DEV), X.to(DEV), out, st)
     torch.cuda.synchronize()
@@ -118,6 +118,51 @@ def test_grad_gemms_random(M, K, V):
     assert_bf16_close(gpu_dx(dl, W, torch.bfloat16), refx, "dX BF16", abs_tol=gemm_tol(V, dl, W))
     assert_bf16_close(gpu_dw(dl, X, torch.bfloat16), refw, "dW BF16", abs_tol=gemm_tol(M, dl, X))
     assert torch.equal(dX, gpu_dx(dl, W)) and torch.equal(dW, gpu_dw(dl, X))
+
+
+def _dx_split_tiles(M, K):
+    """Tiles of lmhead_bwd_dx split into two k-halves: with 256 x 256 CTA-pair
+    tiles on (SMs / 2) pairs, a last wave of rem tiles with 2 rem <= pairs."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tiles, pairs = (-(-K // 256)) * (-(-M // 256)), sms // 2
+    rem = tiles % pairs
+    return rem if tiles > pairs and 0 < 2 * rem <= pairs else 0
+
+
+def test_dx_last_wave_split_integer_exact():
+    """2560 tokens x K = 2048: 80 pair tiles, so on 74 SM pairs the last 6 are
+    computed as two k-halves added into zeroed output.  Integer operands keep
+    every partial sum exact, so the words must equal the oracle's; V = 1032
+    gives 17 k-blocks (halves of 8 and 9, the last one ragged)."""
+    M, K, V = 2560, 2048, 1032
+    if _dx_split_tiles(M, K) == 0:
+        pytest.skip("this GPU's SM count does not split the last wave of this shape")
+    dl = synth.int_bf16((M, V), 51)
+    W = synth.int_bf16((V, K), 52)
+    dX = gpu_dx(dl, W)
+    ref = oracle.round_f32(oracle.dx(bits(dl), bits(W)))
+    got = dX.cpu().numpy()
+    assert np.array_equal(got, ref)  # -0.0 == +0.0: a split sum of 0 is +0
+    assert torch.equal(dX, gpu_dx(dl, W))
+
+
+def test_dx_last_wave_split_random_deterministic():
+    M, K, V = 2560, 2048, 1032
+    if _dx_split_tiles(M, K) == 0:
+        pytest.skip("this GPU's SM count does not split the last wave of this shape")
+    dl = synth.normal_bf16((M, V), 1e-3, 53)
+    W = synth.normal_bf16((V, K), 0.02, 54)
+    # garbage in the output beforehand: the call zeroes the rows it adds into
+    out = guarded_full((M, K), float("nan"))
+    st = status_word()
+    lmhead.lmhead_bwd_dx(dl.to(DEV), W.to(DEV), out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = np.unique(np.concatenate([np.arange(0, M, 97), np.arange(M - 300, M)]))
+    assert_abs_close(to_f64(out[torch.as_tensor(rows, device=DEV)]),
+                     oracle.dx(bits(dl), bits(W), rows=rows), gemm_tol(V, dl, W), "dX split")
+    for _ in range(3):
+        assert torch.equal(out, gpu_dx(dl, W))
 
 
 def test_grad_gemms_large_sampled():

@@ -3,6 +3,10 @@
 * A bounded pipeline wait is made to run out on purpose (a barrier nothing
   arrives at): the kernel unwinds, reports LMH_DEV_PIPE_TIMEOUT through the
   status word, and the context stays usable.  No fault, trap or hang.
+* The same for the vocabulary GEMM itself: with every pipeline wait limited
+  to 1 ns its waits run out, each CTA lets its issued operand copies land,
+  drains its MMAs, frees tensor memory and sets the status bit; the next
+  normal call on the same buffers is bit-exact.
 * The whole five-call step is captured in a CUDA graph and replayed: the calls
   only enqueue stream work (no allocation, no synchronisation), and replays
   reproduce the eager results bit for bit.
@@ -11,6 +15,7 @@ import pytest
 import torch
 
 from lm_head_fp32_b200 import lmhead, synth
+from helpers import guarded_empty, guarded_full
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -24,12 +29,34 @@ def test_watchdog_wait_runs_out_and_context_survives():
     # the context is still usable: a normal call afterwards succeeds
     X = synth.int_bf16((16, 64), 1)
     W = synth.int_bf16((256, 64), 2)
-    out = torch.empty((16, 256), dtype=torch.float32, device=DEV)
+    out = guarded_empty((16, 256), torch.float32)
     st2 = torch.zeros(1, dtype=torch.int32, device=DEV)
     lmhead.lmhead_fwd(X.to(DEV), W.to(DEV), out, st2)
     torch.cuda.synchronize()
     assert int(st2.item()) == 0
     ref = (X.to(torch.int64) @ W.to(torch.int64).T).to(torch.float32)
+    assert torch.equal(out.cpu(), ref)
+
+
+def test_gemm_wait_runs_out_unwinds_and_next_call_is_exact():
+    # 64 tokens: single-CTA tiles (two CTAs resident per SM, one tile each);
+    # a tile's mainloop over K = 8192 takes tens of microseconds, far beyond a
+    # 1 ns limit, so the epilogue's first wait for its accumulator runs out
+    M, K, V = 64, 8192, 32768
+    X = synth.int_bf16((M, K), 11)
+    W = synth.int_bf16((V, K), 12)
+    Xd, Wd = X.to(DEV), W.to(DEV)
+    out = guarded_full((M, V), float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    lmhead.gemm_watchdog_selftest(Xd, Wd, out, status, limit_ns=1)
+    torch.cuda.synchronize()
+    assert int(status.item()) & lmhead.DEV_PIPE_TIMEOUT
+    st2 = torch.zeros(1, dtype=torch.int32, device=DEV)
+    lmhead.lmhead_fwd(Xd, Wd, out, st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0
+    # integers in [-8, 8] with K * 64 < 2^24: every partial sum is exact
+    ref = (X.double() @ W.double().T).to(torch.float32)
     assert torch.equal(out.cpu(), ref)
 
 
@@ -40,9 +67,9 @@ def test_whole_step_in_a_cuda_graph():
     Xd, Wd, td = X.to(DEV), W.to(DEV), t.to(DEV)
     g = torch.tensor([cfg.grad_scalar(t)], dtype=torch.float32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    bufs = dict(logits=torch.empty((M, V), device=DEV), stats=torch.empty((M, 4), device=DEV),
-                dl=torch.empty((M, V), dtype=torch.bfloat16, device=DEV),
-                dX=torch.empty((M, K), device=DEV), dW=torch.empty((V, K), device=DEV))
+    bufs = dict(logits=guarded_empty((M, V)), stats=guarded_empty((M, 4)),
+                dl=guarded_empty((M, V), torch.bfloat16),
+                dX=guarded_empty((M, K)), dW=guarded_empty((V, K)))
 
     def step():
         lmhead.lmhead_fwd(Xd, Wd, bufs["logits"], status)

@@ -1,5 +1,6 @@
-"""The exchange logic of the vocabulary-parallel step on CPU: two gloo ranks,
-each holding one shard of the vocabulary, run vocab_parallel.step with
+"""The exchange logic of the vocabulary-parallel step on CPU: two or three gloo
+ranks, each holding one shard of the vocabulary (possibly an empty one), run
+vocab_parallel.step with
 float64 stand-ins for the CUDA calls (same contracts as include/lmhead.h);
 the merged statistics, the all-reduced dX and the per-rank dW rows must equal
 the whole-vocabulary oracle."""
@@ -12,68 +13,14 @@ import pytest
 import torch
 import torch.multiprocessing as mp
 
+from helpers import FakeOps
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-class FakeOps:
-    """float64 restatement of the library calls' contracts, on CPU tensors."""
-
-    @staticmethod
-    def lmhead_fwd(X, W, out, status=None):
-        out.copy_((X.double() @ W.double().T).float())
-
-    @staticmethod
-    def ce_fwd_shard(logits, target, rec, off, vtot, ignore, status=None):
-        x = logits.double().numpy()
-        V = x.shape[1]
-        r = np.zeros((x.shape[0], 4))
-        for i, y in enumerate(target.tolist()):
-            if y == ignore or y < 0 or y >= vtot:
-                continue
-            m = x[i].max()
-            own = off <= y < off + V
-            r[i] = (m, np.exp(x[i] - m).sum(), x[i, y - off] if own else 0.0, 1.0 if own else 0.0)
-        rec.copy_(torch.from_numpy(r).float())
-
-    @staticmethod
-    def ce_merge_shards(recs, target, stats, vtot, ignore, status=None):
-        R = recs.double().numpy()
-        out = np.zeros((R.shape[1], 4))
-        for i, y in enumerate(target.tolist()):
-            if y == ignore or y < 0 or y >= vtot:
-                continue
-            m = R[:, i, 0].max()
-            d = (R[:, i, 1] * np.exp(R[:, i, 0] - m)).sum()
-            xy = R[R[:, i, 3] != 0, i, 2].sum()
-            out[i] = (m, d, xy, m + np.log(d) - xy)
-        stats.copy_(torch.from_numpy(out).float())
-
-    @staticmethod
-    def ce_bwd_shard(logits, target, stats, g, dl, off, vtot, ignore, status=None):
-        x = logits.double().numpy()
-        st = stats.double().numpy()
-        out = np.zeros_like(x)
-        for i, y in enumerate(target.tolist()):
-            if y == ignore or y < 0 or y >= vtot:
-                continue
-            out[i] = np.exp(x[i] - st[i, 0]) / st[i, 1]
-            if off <= y < off + x.shape[1]:
-                out[i, y - off] -= 1.0
-            out[i] *= float(g.reshape(-1)[0])
-        dl.copy_(torch.from_numpy(out).to(dl.dtype))
-
-    @staticmethod
-    def lmhead_bwd_dx(dl, W, dX, status=None):
-        dX.copy_((dl.double() @ W.double()).float())
-
-    @staticmethod
-    def lmhead_bwd_dw(dl, X, dW, status=None):
-        dW.copy_((dl.double().T @ X.double()).float())
-
-
-def _inputs():
+def _inputs(V=40):
     g = torch.Generator().manual_seed(5)
-    M, K, V = 12, 16, 40
+    M, K = 12, 16
     X = (torch.randn(M, K, generator=g)).to(torch.bfloat16)
     W = (torch.randn(V, K, generator=g) * 0.3).to(torch.bfloat16)
     t = torch.randint(0, V, (M,), generator=g)
@@ -81,14 +28,14 @@ def _inputs():
     return X, W, t, V
 
 
-def _rank(rank, world, port, q):
+def _rank(rank, world, port, q, V=40):
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
                       MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
     from lm_head_fp32_b200 import vocab_parallel
     dist.init_process_group("gloo", rank=rank, world_size=world)
-    X, W, t, V = _inputs()
+    X, W, t, V = _inputs(V)
     off, n = vocab_parallel.shard_bounds(V, world, rank)
     g = torch.tensor([0.5])
     stats, dX, dW, _, _ = vocab_parallel.step(X, W[off:off + n].contiguous(), t, off, V, g,
@@ -97,22 +44,30 @@ def _rank(rank, world, port, q):
     dist.destroy_process_group()
 
 
-def test_two_ranks_match_whole_vocabulary():
-    import oracle
+def _run_ranks(world, V):
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q, V)) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=120) for _ in range(2)]
+    res = [q.get(timeout=120) for _ in range(world)]
     for p in procs:
         p.join(timeout=60)
     assert all(p.exitcode == 0 for p in procs)
     res.sort(key=lambda r: r[0])
-    X, W, t, V = _inputs()
+    return res
+
+
+@pytest.mark.parametrize("world,V", [(2, 40), (3, 16)])
+def test_ranks_match_whole_vocabulary(world, V):
+    """(3, 16): shards of 8, 8 and 0 entries -- the last rank holds no
+    vocabulary and must still join both collectives."""
+    import oracle
+    res = _run_ranks(world, V)
+    X, W, t, V = _inputs(V)
     L = oracle.logits(X.view(torch.int16).numpy().view(np.uint16),
                       W.view(torch.int16).numpy().view(np.uint16))
     Lf = oracle.round_f32(L)
@@ -129,9 +84,13 @@ def test_two_ranks_match_whole_vocabulary():
 
 def test_shard_bounds_cover_the_vocabulary():
     from lm_head_fp32_b200 import vocab_parallel
-    for V in (40, 128256, 151936, 7):
+    for V in (40, 128256, 151936, 7, 16):
         for world in (1, 2, 3, 8):
             spans = [vocab_parallel.shard_bounds(V, world, r) for r in range(world)]
             assert spans[0][0] == 0 and sum(n for _, n in spans) == V
             for (o1, n1), (o2, _) in zip(spans, spans[1:]):
                 assert o1 + n1 == o2
+            assert all(n >= 0 for _, n in spans)
+    # small vocabularies leave trailing ranks empty (handled by step())
+    assert [vocab_parallel.shard_bounds(16, 3, r)[1] for r in range(3)] == [8, 8, 0]
+    assert [vocab_parallel.shard_bounds(40, 8, r)[1] for r in range(8)] == [8] * 5 + [0] * 3

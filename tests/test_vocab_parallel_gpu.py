@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from lm_head_fp32_b200 import lmhead, synth, vocab_parallel
-from helpers import assert_abs_close, assert_bf16_close, bits, gemm_tol, loss_tol, to_f64
+from helpers import assert_abs_close, assert_bf16_close, bits, gemm_tol, guarded_empty, loss_tol, to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -34,17 +34,17 @@ def test_shards_match_whole_vocabulary():
     recs, logits = [], []
     for off, n in bounds:
         Wr = W[off:off + n].contiguous().to(DEV)
-        lr = torch.empty((M, n), device=DEV)
+        lr = guarded_empty((M, n))
         lmhead.lmhead_fwd(Xd, Wr, lr, status)
-        rec = torch.empty((M, 4), device=DEV)
+        rec = guarded_empty((M, 4))
         lmhead.ce_fwd_shard(lr, td, rec, off, V, -100, status)
         recs.append(rec)
         logits.append(lr)
-    stats = torch.empty((M, 4), device=DEV)
+    stats = guarded_empty((M, 4))
     lmhead.ce_merge_shards(torch.stack(recs).contiguous(), td, stats, V, -100, status)
     dls = []
     for (off, n), lr in zip(bounds, logits):
-        dl = torch.empty((M, n), dtype=torch.bfloat16, device=DEV)
+        dl = guarded_empty((M, n), torch.bfloat16)
         lmhead.ce_bwd_shard(lr, td, stats, g, dl, off, V, -100, status)
         dls.append(dl)
     torch.cuda.synchronize()
@@ -58,7 +58,7 @@ def test_shards_match_whole_vocabulary():
     assert_abs_close(got[:, 3], ref[:, 3], loss_tol(ref[:, 3]), "merged loss")
     assert (got[~valid] == 0).all()
     # and against the single-device ce_fwd
-    one = torch.empty((M, 4), device=DEV)
+    one = guarded_empty((M, 4))
     lmhead.ce_fwd(full.contiguous(), td, one, -100)
     torch.cuda.synchronize()
     assert_abs_close(got[:, 3], one.cpu().double().numpy()[:, 3], 2 * loss_tol(ref[:, 3]), "vs ce_fwd")
@@ -68,7 +68,7 @@ def test_shards_match_whole_vocabulary():
     # dX = sum over shards, dW = per-shard rows
     dX = torch.zeros((M, K), device=DEV)
     for (off, n), dl in zip(bounds, dls):
-        part = torch.empty((M, K), device=DEV)
+        part = guarded_empty((M, K))
         lmhead.lmhead_bwd_dx(dl, W[off:off + n].contiguous().to(DEV), part)
         dX += part
     dlb = bits(dl_full)
@@ -81,11 +81,11 @@ def test_step_on_one_device_equals_five_calls():
     g = torch.tensor([0.25], device=DEV)
     stats, dX, dW, logits, dl = vocab_parallel.step(Xd, Wd, td, 0, V, g)
     M, K = X.shape
-    ref_l = torch.empty((M, V), device=DEV)
+    ref_l = guarded_empty((M, V))
     lmhead.lmhead_fwd(Xd, Wd, ref_l)
-    ref_s = torch.empty((M, 4), device=DEV)
+    ref_s = guarded_empty((M, 4))
     lmhead.ce_fwd(ref_l, td, ref_s)
-    ref_dl = torch.empty((M, V), dtype=torch.bfloat16, device=DEV)
+    ref_dl = guarded_empty((M, V), torch.bfloat16)
     lmhead.ce_bwd(ref_l, td, ref_s, g, ref_dl)
     torch.cuda.synchronize()
     assert torch.equal(logits, ref_l)
