@@ -59,6 +59,7 @@ struct GemmParams {
     int32_t num_m_tiles;
     int32_t num_n_tiles;
     int32_t m_fastest;  // tile order: 1 = consecutive tiles share n (B panel)
+    int32_t group_m;    // > 0: tiles in groups of group_m m-tiles, m fastest inside a group
     int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
     int32_t l2_b;
     int32_t l2_out;     // L2 policy of the output stores (TMA store epilogue): 0 none, 1 evict first
@@ -170,9 +171,19 @@ __device__ __forceinline__ void stage_out(__nv_bfloat16 *p, uint32_t bits)
     *p = __float2bfloat16_rn(__uint_as_float(bits));
 }
 
-__device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &mt, int &nt)
+__host__ __device__ inline void tile_coords(int t, const GemmParams &p, int &mt, int &nt)
 {
-    if (p.m_fastest) {
+    if (p.group_m > 0) {
+        // groups of group_m m-tiles (the last one possibly narrower), each
+        // swept over every n-tile with m fastest: the tiles running at the
+        // same time share fewer operand panels than a full m sweep would
+        const int span = p.group_m * p.num_n_tiles;
+        const int g = t / span, r = t % span;
+        const int rest = p.num_m_tiles - g * p.group_m;
+        const int gm = rest < p.group_m ? rest : p.group_m;
+        mt = g * p.group_m + r % gm;
+        nt = r / gm;
+    } else if (p.m_fastest) {
         mt = t % p.num_m_tiles;
         nt = t / p.num_m_tiles;
     } else {

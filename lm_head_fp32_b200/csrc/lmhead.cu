@@ -205,14 +205,22 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
         // A last wave of rem tiles on `units` SMs (pairs) that would leave
         // more than half of them idle: split those tiles into two k-halves
         // that both add into zeroed output (deterministic: two addends).
-        // With tiles in m-fastest order they are the last n-rows of the
-        // output, which are contiguous, so one memset zeroes them.
+        // They come last in the tile order, and whole output rows are
+        // contiguous, so one memset zeroes them.
         const int64_t rem = tiles % units;
         const int64_t num_kb = (p.Kdim + lmh::kBlockK - 1) / lmh::kBlockK;
-        if (p.allow_split && p.m_fastest && tiles > units && rem > 0 && 2 * rem <= units &&
-            num_kb >= 2) {
+        if (p.allow_split && (p.m_fastest || p.group_m > 0) && tiles > units && rem > 0 &&
+            2 * rem <= units && num_kb >= 2) {
+            // zero every output row from the lowest n-row any split tile
+            // covers (rows below it are all stored, not added)
             p.split_tiles = static_cast<int32_t>(rem);
-            const int64_t row0 = ((tiles - rem) / p.num_m_tiles) * BN;
+            int nt_min = p.num_n_tiles;
+            for (int64_t t = tiles - rem; t < tiles; ++t) {
+                int mt = 0, nt = 0;
+                lmh::tile_coords(static_cast<int>(t), p, mt, nt);
+                nt_min = nt < nt_min ? nt : nt_min;
+            }
+            const int64_t row0 = static_cast<int64_t>(nt_min) * BN;
             const size_t bytes = static_cast<size_t>(p.Ndim - row0) * p.ldo * sizeof(float);
             if (cudaMemsetAsync(static_cast<float *>(p.out) + row0 * p.ldo, 0, bytes, stream) !=
                 cudaSuccess)
@@ -275,6 +283,14 @@ int pick_bn_tokens(int64_t M)
 #define LMH_LOGITS_L2_POLICY 1
 #endif
 constexpr int kLogitsL2Policy = LMH_LOGITS_L2_POLICY;
+
+// Tile order of dX: groups of this many 256-wide m-tiles (K columns), each
+// swept over every token tile; 0 = all m-tiles first (one W column strip
+// each), the plain m-fastest order.
+#ifndef LMH_DX_GROUP_M
+#define LMH_DX_GROUP_M 0
+#endif
+constexpr int kDxGroupM = LMH_DX_GROUP_M;
 
 // L2 policy of W in the vocabulary GEMM: streamed once (evict first) when a
 // single token tile reads each W panel, normal when several token tiles reuse
@@ -509,6 +525,7 @@ lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(V);
     p.m_fastest = 1;
+    p.group_m = kDxGroupM;
     p.l2_a = 0;  // every W and dlogits chunk is read by the concurrently running tiles
     p.l2_b = 0;
     p.status = status;

@@ -67,9 +67,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait limit of every pipeline wait.  A legitimate wait in these kernels lasts
 // microseconds; after this long the kernel reports a timeout and unwinds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Limits below this are kept by polling with the non-blocking test_wait:
+// try_wait may suspend the thread until the phase completes, which can
+// outlast a short limit many times over.
+constexpr uint64_t kPollLimitNs = 100000ull;
 
 // Wait for the phase of `bar` with the given parity to complete.  Returns
 // false (and sets *abort) when the wait limit passes or when another role of
@@ -78,6 +96,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
                                           uint64_t limit_ns = kWaitLimitNs)
 {
     const uint32_t a = smem_u32(bar);
+    if (limit_ns < kPollLimitNs) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_test_wait(a, parity)) {
+            if (*abort)
+                return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                *abort = 1;
+                return false;
+            }
+        }
+        return true;
+    }
     if (mbar_try_wait(a, parity))
         return true;
     const uint64_t t0 = global_timer_ns();

@@ -120,6 +120,24 @@ def test_grad_gemms_random(M, K, V):
     assert torch.equal(dX, gpu_dx(dl, W)) and torch.equal(dW, gpu_dw(dl, X))
 
 
+@pytest.mark.parametrize("M", [128, 1024])
+def test_sweep_corner_k16384_sampled(M):
+    """The FP32- versus BF16-output sweep's K = 16384 shapes at full size, on
+    the sweep's own inputs (X ~ N(0,1), W ~ N(0,0.02^2), 32768 vocabulary
+    rows): 128 tokens take the single-token-tile CTA-pair path, 1024 tokens
+    the 256 x 256 pair tiles.  Sampled token rows, FP32 and BF16 outputs."""
+    c = next(c for c in synth.sweep_configs() if c.M == M and c.K == 16384)
+    X = synth.normal_bf16((c.M, c.K), 1.0, c.seed)
+    W = synth.normal_bf16((c.V, c.K), 0.02, c.seed + 1)
+    out = gpu_logits(X, W)
+    out16 = gpu_logits(X, W, torch.bfloat16)
+    rows = np.array([0, 1, M // 2 + 3, M - 1])
+    ref = oracle.logits(bits(X), bits(W), rows=rows)
+    tr = torch.as_tensor(rows, device=DEV)
+    assert_abs_close(out[tr].cpu().double().numpy(), ref, logits_tol(X, W), "FP32 logits")
+    assert_bf16_close(out16[tr], ref, "BF16 logits", abs_tol=logits_tol(X, W))
+
+
 def _dx_split_tiles(M, K):
     """Tiles of lmhead_bwd_dx split into two k-halves: with 256 x 256 CTA-pair
     tiles on (SMs / 2) pairs, a last wave of rem tiles with 2 rem <= pairs."""
