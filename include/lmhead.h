@@ -213,7 +213,11 @@ LMH_API lmh_status_t ce_bwd_shard(const float *logits, const int64_t *target, co
  *   dlogits [M,V] BF16.  W [V,K] BF16.
  *   dX      [M,K] FP32 (LMH_F32) or BF16 (LMH_BF16).
  *   Requirements: V % 8 == 0 and K % 8 == 0 (16-byte rows), inputs 16-byte
- *   aligned.  Deterministic. */
+ *   aligned.  Deterministic.  With an FP32 dX the output tiles of a last
+ *   wave that would leave most SMs idle are computed as two halves of the
+ *   reduction that are both added into rows of dX the call first zeroes on
+ *   the stream; with two addends the order of the additions does not change
+ *   the result. */
 LMH_API lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t out_dtype,
                            int64_t M, int64_t K, int64_t V, int32_t *status,
                            lmh_stream_t stream);

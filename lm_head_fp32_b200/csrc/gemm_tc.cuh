@@ -59,18 +59,17 @@ struct GemmParams {
     int32_t num_m_tiles;
     int32_t num_n_tiles;
     int32_t m_fastest;  // tile order: 1 = consecutive tiles share n (B panel)
-    int32_t group_m;    // > 0: tiles in groups of group_m m-tiles, m fastest inside a group
     int32_t l2_a;       // L2 policy of A / B loads: 0 normal, 1 evict first, 2 evict last
     int32_t l2_b;
     int32_t l2_out;     // L2 policy of the output stores (TMA store epilogue): 0 none, 1 evict first
     int32_t *status;
     uint64_t wait_limit_ns;  // limit of every pipeline wait (the host sets kWaitLimitNs)
     // The last split_tiles tiles of the tile order are each computed as two
-    // work items, the first and the second half of the k-blocks, whose FP32
-    // sums are both added (TMA reduce-add) into output the host has zeroed:
-    // fl(0 + a) = a and fl(a + b) = fl(b + a), so the result does not depend on
-    // which half lands first.  Used for a last wave that would leave most
-    // SMs idle; 0 = no split (requires two or more k-blocks).
+    // work items, the first and the second half of the k-blocks (all first
+    // halves, then all second halves), whose FP32 sums are both added (TMA
+    // reduce-add) into output the host has zeroed: fl(0 + a) = a and
+    // fl(a + b) = fl(b + a), so the result does not depend on which half lands
+    // first.  0 = no split (requires two or more k-blocks).
     int32_t split_tiles;
     int32_t allow_split;  // host side: the call may split its last wave (FP32 output)
     // fused cross-entropy statistics (vocabulary GEMM only): per 128-wide
@@ -173,17 +172,7 @@ __device__ __forceinline__ void stage_out(__nv_bfloat16 *p, uint32_t bits)
 
 __host__ __device__ inline void tile_coords(int t, const GemmParams &p, int &mt, int &nt)
 {
-    if (p.group_m > 0) {
-        // groups of group_m m-tiles (the last one possibly narrower), each
-        // swept over every n-tile with m fastest: the tiles running at the
-        // same time share fewer operand panels than a full m sweep would
-        const int span = p.group_m * p.num_n_tiles;
-        const int g = t / span, r = t % span;
-        const int rest = p.num_m_tiles - g * p.group_m;
-        const int gm = rest < p.group_m ? rest : p.group_m;
-        mt = g * p.group_m + r % gm;
-        nt = r / gm;
-    } else if (p.m_fastest) {
+    if (p.m_fastest) {
         mt = t % p.num_m_tiles;
         nt = t / p.num_m_tiles;
     } else {
@@ -290,10 +279,13 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
             kb1 = num_kb;
             return false;
         }
+        // every split tile's first half, then every second half (all of them
+        // run in the same wave)
         const int j = it - split_first;
-        t = split_first + (j >> 1);
-        kb0 = (j & 1) ? num_kb / 2 : 0;
-        kb1 = (j & 1) ? num_kb : num_kb / 2;
+        const bool second = j >= p.split_tiles;
+        t = split_first + (second ? j - p.split_tiles : j);
+        kb0 = second ? num_kb / 2 : 0;
+        kb1 = second ? num_kb : num_kb / 2;
         return true;
     };
 

@@ -23,6 +23,7 @@ constexpr int64_t kMaxDim = 0x7fffffff;
 constexpr int kMaxDevices = 64;
 constexpr int kCeThreads = 1024;  // threads per cross-entropy CTA; one CTA per row
 
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int num_sms()
@@ -201,21 +202,25 @@ lmh_status_t launch_gemm_impl(const CUtensorMap &ta, const CUtensorMap &tb, cons
     // persistent: one CTA (or CTA pair) per SM (pair); several resident per SM: one per tile
     const int64_t units = RES == 1 ? num_sms() / C::CTAS : tiles;
     p.split_tiles = 0;
-    if constexpr (TMA_STORE && sizeof(OutT) == 4 && !CE && !ACC && RES == 1) {
-        // A last wave of rem tiles on `units` SMs (pairs) that would leave
-        // more than half of them idle: split those tiles into two k-halves
-        // that both add into zeroed output (deterministic: two addends).
-        // They come last in the tile order, and whole output rows are
-        // contiguous, so one memset zeroes them.
+    if constexpr (sizeof(OutT) == 4 && !CE && !ACC && RES == 1) {
+        // A last (or only) wave of rem tiles that would leave more than half
+        // of the SMs (pairs) idle: split those tiles into two k-halves that
+        // both add into zeroed output (TMA reduce-add, or per-element atomic
+        // adds on the direct-store path; deterministic: two addends, so both
+        // epilogue paths give the same bits).  The split tiles come last in
+        // the tile order, and whole output rows are contiguous, so one memset
+        // zeroes them.
         const int64_t rem = tiles % units;
         const int64_t num_kb = (p.Kdim + lmh::kBlockK - 1) / lmh::kBlockK;
-        if (p.allow_split && (p.m_fastest || p.group_m > 0) && tiles > units && rem > 0 &&
-            2 * rem <= units && num_kb >= 2) {
+        int64_t split = 0;
+        if (p.allow_split && p.m_fastest && num_kb >= 2 && rem > 0 && 2 * rem <= units)
+            split = rem;
+        if (split > 0) {
             // zero every output row from the lowest n-row any split tile
             // covers (rows below it are all stored, not added)
-            p.split_tiles = static_cast<int32_t>(rem);
+            p.split_tiles = static_cast<int32_t>(split);
             int nt_min = p.num_n_tiles;
-            for (int64_t t = tiles - rem; t < tiles; ++t) {
+            for (int64_t t = tiles - split; t < tiles; ++t) {
                 int mt = 0, nt = 0;
                 lmh::tile_coords(static_cast<int>(t), p, mt, nt);
                 nt_min = nt < nt_min ? nt : nt_min;
@@ -283,14 +288,6 @@ int pick_bn_tokens(int64_t M)
 #define LMH_LOGITS_L2_POLICY 1
 #endif
 constexpr int kLogitsL2Policy = LMH_LOGITS_L2_POLICY;
-
-// Tile order of dX: groups of this many 256-wide m-tiles (K columns), each
-// swept over every token tile; 0 = all m-tiles first (one W column strip
-// each), the plain m-fastest order.
-#ifndef LMH_DX_GROUP_M
-#define LMH_DX_GROUP_M 0
-#endif
-constexpr int kDxGroupM = LMH_DX_GROUP_M;
 
 // L2 policy of W in the vocabulary GEMM: streamed once (evict first) when a
 // single token tile reads each W panel, normal when several token tiles reuse
@@ -525,7 +522,6 @@ lmh_status_t lmhead_bwd_dx(const void *dlogits, const void *W, void *dX, int32_t
     p.Ndim = static_cast<int32_t>(M);
     p.Kdim = static_cast<int32_t>(V);
     p.m_fastest = 1;
-    p.group_m = kDxGroupM;
     p.l2_a = 0;  // every W and dlogits chunk is read by the concurrently running tiles
     p.l2_b = 0;
     p.status = status;

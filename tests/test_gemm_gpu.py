@@ -138,13 +138,14 @@ def test_sweep_corner_k16384_sampled(M):
     assert_bf16_close(out16[tr], ref, "BF16 logits", abs_tol=logits_tol(X, W))
 
 
-def _dx_split_tiles(M, K):
-    """Tiles of lmhead_bwd_dx split into two k-halves: with 256 x 256 CTA-pair
-    tiles on (SMs / 2) pairs, a last wave of rem tiles with 2 rem <= pairs."""
+def _dx_split_tiles(M, K, V):
+    """Tiles of lmhead_bwd_dx split into two k-halves, as the library decides
+    for 256 x 256 CTA-pair tiles on (SMs / 2) pairs: those of a last (or only)
+    wave that fills at most half of the pairs."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles, pairs = (-(-K // 256)) * (-(-M // 256)), sms // 2
     rem = tiles % pairs
-    return rem if tiles > pairs and 0 < 2 * rem <= pairs else 0
+    return rem if 0 < 2 * rem <= pairs else 0
 
 
 def test_dx_last_wave_split_integer_exact():
@@ -153,7 +154,7 @@ def test_dx_last_wave_split_integer_exact():
     every partial sum exact, so the words must equal the oracle's; V = 1032
     gives 17 k-blocks (halves of 8 and 9, the last one ragged)."""
     M, K, V = 2560, 2048, 1032
-    if _dx_split_tiles(M, K) == 0:
+    if _dx_split_tiles(M, K, V) == 0:
         pytest.skip("this GPU's SM count does not split the last wave of this shape")
     dl = synth.int_bf16((M, V), 51)
     W = synth.int_bf16((V, K), 52)
@@ -166,7 +167,7 @@ def test_dx_last_wave_split_integer_exact():
 
 def test_dx_last_wave_split_random_deterministic():
     M, K, V = 2560, 2048, 1032
-    if _dx_split_tiles(M, K) == 0:
+    if _dx_split_tiles(M, K, V) == 0:
         pytest.skip("this GPU's SM count does not split the last wave of this shape")
     dl = synth.normal_bf16((M, V), 1e-3, 53)
     W = synth.normal_bf16((V, K), 0.02, 54)
@@ -180,6 +181,28 @@ def test_dx_last_wave_split_random_deterministic():
     assert_abs_close(to_f64(out[torch.as_tensor(rows, device=DEV)]),
                      oracle.dx(bits(dl), bits(W), rows=rows), gemm_tol(V, dl, W), "dX split")
     for _ in range(3):
+        assert torch.equal(out, gpu_dx(dl, W))
+
+
+def test_dx_single_sparse_wave_split_integer_exact_and_deterministic():
+    """Few tiles (a ragged token tile, 384 = 256 + 128, and K = 256: two pair
+    tiles) on many SM pairs: both tiles are split into k-halves, so four pairs
+    work.  V = 65544 gives 1025 k-blocks (halves of 512 and 513, the last one
+    ragged).  Integer operands keep the words exact; random operands are within
+    the tolerance and bitwise repeatable."""
+    M, K, V = 384, 256, 65544
+    assert _dx_split_tiles(M, K, V) == 2
+    dl = synth.int_bf16((M, V), 61)
+    W = synth.int_bf16((V, K), 62)
+    got = gpu_dx(dl, W).cpu().numpy()
+    assert np.array_equal(got, oracle.round_f32(oracle.dx(bits(dl), bits(W))))
+    dl = synth.normal_bf16((M, V), 1e-3, 63)
+    W = synth.normal_bf16((V, K), 0.02, 64)
+    out = gpu_dx(dl, W)
+    rows = np.array([0, 1, 200, 255, 256, 300, M - 1])
+    assert_abs_close(to_f64(out[torch.as_tensor(rows, device=DEV)]),
+                     oracle.dx(bits(dl), bits(W), rows=rows), gemm_tol(V, dl, W), "dX split")
+    for _ in range(2):
         assert torch.equal(out, gpu_dx(dl, W))
 
 
@@ -202,7 +225,8 @@ def test_grad_gemms_large_sampled():
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_direct_store_epilogue_on_unaligned_output(dtype):
     """An output a tensor map cannot describe (base not 16-byte aligned) takes
-    the direct-store epilogue; the results are the same bits."""
+    the direct-store epilogue; the results are the same bits (dX here has
+    three tiles, split into k-halves on both paths)."""
     M, K, V = 70, 264, 1000
     X = synth.normal_bf16((M, K), 1.0, 5)
     W = synth.normal_bf16((V, K), 0.02, 6)
