@@ -83,7 +83,10 @@ struct GemmParams {
 };
 
 constexpr int kEpiSlots = 8;  // 32 x EPI_CHUNK staging slots shared by the epilogue warps
-constexpr unsigned kDwStorePaceNs = 200;  // pause after each dW sub-tile store
+#ifndef LMH_DW_STORE_PACE_NS
+#define LMH_DW_STORE_PACE_NS 200
+#endif
+constexpr unsigned kDwStorePaceNs = LMH_DW_STORE_PACE_NS;  // pause after each dW sub-tile store
 
 // Epilogue warps of each GEMM.  Measured at 1024 x 4096 x 32768 (L2 flushed,
 // medians): eight take the fused cross-entropy GEMM from 195.6 to 187.4 us,
@@ -528,7 +531,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                         // output; spacing the sub-tile stores keeps them from
                         // delaying the operand loads queued behind them
                         // (measured 214.0 -> 206.9 us at 1024 x 4096 x 32768)
-                        __nanosleep(kDwStorePaceNs);
+                        if (kDwStorePaceNs > 0)
+                            __nanosleep(kDwStorePaceNs);
                     }
                     if constexpr (CE) {
                         // the TMA store only reads the slot, so it can be read here too
