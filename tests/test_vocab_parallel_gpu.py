@@ -100,3 +100,32 @@ def test_step_on_one_device_equals_five_calls():
     lmhead.lmhead_bwd_dw(ref_dl, Xd, ref_dw)
     torch.cuda.synchronize()
     assert torch.equal(dX, ref_dx) and torch.equal(dW, ref_dw)
+
+
+def test_merge_with_an_empty_shard_record():
+    """A rank whose vocabulary shard is empty contributes the neutral record
+    {-inf, 0, 0, 0} (vocab_parallel.step); merging it with the other shards'
+    records must give the same statistics as merging those alone."""
+    X, W, t, V, bounds = _case(M=40, K=64, bounds=((0, 200), (200, 144)), seed=13)
+    M = X.shape[0]
+    Xd, td = X.to(DEV), t.to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    recs = []
+    for off, n in bounds:
+        lr = guarded_empty((M, n))
+        lmhead.lmhead_fwd(Xd, W[off:off + n].contiguous().to(DEV), lr, status)
+        rec = guarded_empty((M, 4))
+        lmhead.ce_fwd_shard(lr, td, rec, off, V, -100, status)
+        recs.append(rec)
+    empty = torch.zeros((M, 4), device=DEV)
+    empty[:, 0] = float("-inf")
+    with_empty = guarded_empty((M, 4))
+    lmhead.ce_merge_shards(torch.stack(recs + [empty]).contiguous(), td, with_empty, V, -100, status)
+    first_empty = guarded_empty((M, 4))
+    lmhead.ce_merge_shards(torch.stack([empty] + recs).contiguous(), td, first_empty, V, -100, status)
+    without = guarded_empty((M, 4))
+    lmhead.ce_merge_shards(torch.stack(recs).contiguous(), td, without, V, -100, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == lmhead.DEV_BAD_TARGET      # only the planted bad target
+    assert torch.equal(with_empty, without) and torch.equal(first_empty, without)
+    assert bool(torch.isfinite(without).all())
