@@ -67,9 +67,10 @@ struct GemmParams {
     // The last split_tiles tiles of the tile order are each computed as two
     // work items, the first and the second half of the k-blocks (all first
     // halves, then all second halves), whose FP32 sums are both added (TMA
-    // reduce-add) into output the host has zeroed: fl(0 + a) = a and
-    // fl(a + b) = fl(b + a), so the result does not depend on which half lands
-    // first.  0 = no split (requires two or more k-blocks).
+    // reduce-add, or atomic adds on the direct-store path) into output the
+    // host has zeroed: fl(0 + a) = a and fl(a + b) = fl(b + a), so the result
+    // does not depend on which half lands first.  0 = no split (requires two
+    // or more k-blocks).
     int32_t split_tiles;
     int32_t allow_split;  // host side: the call may split its last wave (FP32 output)
     // fused cross-entropy statistics (vocabulary GEMM only): per 128-wide
@@ -127,7 +128,8 @@ struct GemmCfg {
     static constexpr int XCH_BYTES = CE ? 2 * 3 * 32 * 8 + 4 * 8 : 0;
     // 1024 bytes of alignment slack, the ring (each stage with its full and
     // empty barrier), the staging slots, acc_full[2], acc_empty[2], drain,
-    // the tensor-memory address and abort flag (16), the CE exchange
+    // the tensor-memory address, abort flag and issued k-block count (16),
+    // the CE exchange
     static constexpr int BUDGET = RES == 1 ? kSmemLimit : kSmemPerSm / RES - 1024;
     static constexpr int STAGES_RAW =
         (BUDGET - 1024 - EPI_BYTES - 5 * 8 - 16 - XCH_BYTES) / (STAGE_BYTES + 16);
