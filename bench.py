@@ -573,6 +573,7 @@ def vocab_line(cfg, world: int, steps: int, warmup: int, total_ms: float, stage_
     (strong scaling); total_ms is the maximum over ranks of the summed step
     times, stage_ms this rank's mean time per stage."""
     M, K = cfg.M, cfg.K
+    peak_t, peak_kind = tensor_peak(peaks, clocks)
     flop = 2.0 * M * K * shard_rows
     work = {"lmhead_fwd": ("tensor", flop), "lmhead_bwd_dx": ("tensor", flop),
             "lmhead_bwd_dw": ("tensor", flop),
@@ -585,11 +586,13 @@ def vocab_line(cfg, world: int, steps: int, warmup: int, total_ms: float, stage_
             continue
         bound, w = work[n]
         if bound == "tensor":
-            ach, peak, unit = w / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+            ach, peak, unit = w / (ms / 1e3) / 1e12, peak_t, "TFLOP/s"
         else:
             ach, peak, unit = w / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
         kernels[n] = {"ms": round(ms, 5), "bound": bound, "achieved": round(ach, 1), "unit": unit,
                       "frac": round(ach / peak, 4), "algorithmic": w}
+        if bound == "tensor":
+            kernels[n]["frac_of_burst"] = round(ach / peaks["bf16_tflops"], 4)
     dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["ms"])
     kd = kernels[dom]
     return {"metric": METRIC, "value": M * steps / (total_ms / 1e3), "unit": "tokens/s",
@@ -604,9 +607,10 @@ def vocab_line(cfg, world: int, steps: int, warmup: int, total_ms: float, stage_
                        "step": "lmhead_fwd, ce_fwd_shard, all-gather [M,4], ce_merge_shards, "
                                "ce_bwd_shard, lmhead_bwd_dx, all-reduce dX, lmhead_bwd_dw"},
             "roofline": {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"],
-                         "peak": peaks["bf16_tflops"] if kd["bound"] == "tensor" else peaks["hbm_gbs"],
+                         "peak": peak_t if kd["bound"] == "tensor" else peaks["hbm_gbs"],
                          "unit": kd["unit"], "frac": kd["frac"],
-                         "peak_source": f"{peak_src} (burst)", "traffic": None},
+                         "peak_source": f"{peak_src} ({peak_kind if kd['bound'] == 'tensor' else 'copy'})",
+                         "traffic": None},
             "kernels": kernels, "clocks": clocks}
 
 
