@@ -474,7 +474,7 @@ const char *lmh_status_string(lmh_status_t s)
     return "unknown status";
 }
 
-int32_t lmh_version(void) { return 100; }
+int32_t lmh_version(void) { return 20000; }
 
 lmh_status_t lmh_watchdog_selftest(int32_t *status, int64_t limit_us, lmh_stream_t stream)
 {

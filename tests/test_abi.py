@@ -52,7 +52,7 @@ def test_header_compiles_as_plain_c():
 def test_status_strings_and_version():
     assert lmhead.status_string(0) == "ok"
     assert "misaligned" in lmhead.status_string(2)
-    assert lmhead.lib().lmh_version() >= 100
+    assert lmhead.lib().lmh_version() == 20000      # 2.0.0
 
 
 P = ctypes.c_void_p
