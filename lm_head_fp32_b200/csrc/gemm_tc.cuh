@@ -191,30 +191,46 @@ __host__ __device__ inline void tile_coords(int t, const GemmParams &p, int &mt,
 // columns starting at vbase; columns at or past V excluded) and returns its
 // (max, sum of exp(x - max)); the lane whose row holds its token's target
 // column also records the target logit.  Lanes without a token return the
-// empty pair.  The columns are visited in a lane-rotated order, so the 32
-// lanes read 32 different banks.
+// empty pair.  The row is read as eight 16-byte chunks, lane l starting at
+// chunk l mod 8, so the eight lanes of each quarter-warp read eight different
+// bank groups; max and sum do not depend on the order the values are held in.
 __device__ __forceinline__ MaxSum ce_subtile_stats(const float *buf, int lane, int rows, int vbase,
                                                    int V, int tok, int ntok, const GemmParams &p)
 {
     if (lane >= rows || tok >= ntok)
         return MaxSum{-INFINITY, 0.f};
     const float *rowp = buf + lane * 32;
+    const float4 *row4 = reinterpret_cast<const float4 *>(rowp);
     const int nvalid = V - vbase;  // may be <= 0 (a slice past the vocabulary) or > 32
-    float vmax = -INFINITY;
+    float v[32];
 #pragma unroll
-    for (int kk = 0; kk < 32; ++kk) {
-        const int col = (kk + lane) & 31;
-        if (col < nvalid)
-            vmax = fmaxf(vmax, rowp[col]);
+    for (int kk = 0; kk < 8; ++kk) {
+        const float4 q = row4[(kk + lane) & 7];
+        v[4 * kk + 0] = q.x;
+        v[4 * kk + 1] = q.y;
+        v[4 * kk + 2] = q.z;
+        v[4 * kk + 3] = q.w;
     }
+    if (nvalid < 32) {
+        // the vocabulary ends inside this block (the same for the whole warp)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const int c = (kk + lane) & 7;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (4 * c + e >= nvalid)
+                    v[4 * kk + e] = -INFINITY;
+        }
+    }
+    float vmax = v[0];
+#pragma unroll
+    for (int i = 1; i < 32; ++i)
+        vmax = fmaxf(vmax, v[i]);
     float dsum = 0.f;
     if (vmax != -INFINITY) {
 #pragma unroll
-        for (int kk = 0; kk < 32; ++kk) {
-            const int col = (kk + lane) & 31;
-            if (col < nvalid)
-                dsum += exp_neg(rowp[col] - vmax);
-        }
+        for (int i = 0; i < 32; ++i)
+            dsum += exp_neg(v[i] - vmax);  // a masked column adds exp(-inf) = 0
     }
     const int64_t y = p.ce_target[tok];
     if (y >= vbase && y < vbase + 32 && y < V)
