@@ -230,7 +230,7 @@ __device__ __forceinline__ MaxSum ce_subtile_stats(const float *buf, int lane, i
     if (vmax != -INFINITY) {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            dsum += exp_neg(v[i] - vmax);  // a masked column adds exp(-inf) = 0
+            dsum += exp_neg_ftz(v[i] - vmax);  // a masked column adds exp(-inf) = 0
     }
     const int64_t y = p.ce_target[tok];
     if (y >= vbase && y < vbase + 32 && y < V)
