@@ -101,6 +101,26 @@ def test_ce_bad_target_sets_status_and_zeroes_row():
     check_dl(dl, x, t, 1.0)
 
 
+def test_ce_ignored_rows_are_not_read():
+    """Ignored rows hold NaN here: the kernels never read them (zero statistics
+    and gradient, no status bit), and the other rows are unaffected.  A batch
+    in which every row is ignored gives zeros throughout."""
+    M, V = 70, 3000
+    x, _ = synth.ce_logits(M, V, 4.0, 21)
+    t = synth.targets(M, V, 0.0, 21)
+    t[1::2] = -100
+    x[1::2] = float("nan")
+    st, dl, status = run_ce(x.to(DEV), t.to(DEV), 1.0, torch.bfloat16)
+    assert status == 0
+    assert (st[1::2] == 0).all() and (dl[1::2].float() == 0).all()
+    check_stats(st, x, t)
+    check_dl(dl, x, t, 1.0)
+    t[:] = -100
+    st, dl, status = run_ce(x.to(DEV), t.to(DEV), 1.0)
+    assert status == 0
+    assert (st == 0).all() and (dl == 0).all()
+
+
 def test_ce_custom_ignore_index_and_per_row_grad():
     M, V = 33, 2048
     x, _ = synth.ce_logits(M, V, 3.0, 8)

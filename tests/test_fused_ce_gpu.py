@@ -93,6 +93,20 @@ def test_fused_ce_bad_targets_and_custom_ignore_index():
     check(X, W, t, ignore=11)
 
 
+def test_fused_ce_every_row_ignored():
+    """Every target is ignore_index: the logits are still those of lmhead_fwd,
+    every statistics row is zero and no status bit is set."""
+    M, K, V = 40, 256, 1000
+    X = synth.normal_bf16((M, K), 1.0, 5)
+    W = synth.normal_bf16((V, K), 0.02, 6)
+    t = torch.full((M,), -100, dtype=torch.int64)
+    lf, sf, st = fused(X, W, t)
+    ls, _, _ = separate(X, W, t)
+    assert st == 0
+    assert torch.equal(lf, ls)
+    assert (sf == 0).all()
+
+
 def test_fused_ce_fallback_paths():
     # V % 4 != 0: the logits cannot go through the TMA-store epilogue, so the call
     # runs the two separate passes; the results still match the oracle
