@@ -112,16 +112,22 @@ void oracle_logits(const uint16_t *X, const uint16_t *W, int64_t M, int64_t K,
 
 /* For one row x[0..V) with target y:
  *   m   = max_j x_j
- *   d   = sum_j exp(x_j - m)
+ *   s   = sum_{j != y} exp(x_j - m)        (the other columns' share)
+ *   d   = s + exp(x_y - m)                 (= sum_j exp(x_j - m))
  *   x_y = x_y
- *   loss = -log softmax(x)_y = m + log(d) - x_y
+ *   loss = -log softmax(x)_y = log(d / exp(x_y - m)) = log1p(s * exp(m - x_y))
+ * The loss is the same value as m + log(d) - x_y, written through s: when the
+ * target holds nearly all of the row's mass, d = 1 + s rounds most of s away
+ * (even in FP64 for s below ~1e-12), and log(d) would lose it.
  * y == ignore_index: the row is ignored (loss 0, stats 0, x not read).
  * y outside [0,V) and not ignore_index: reported as a bad target and
- * treated like an ignored row. */
+ * treated like an ignored row.  *s_out (may be NULL) receives s. */
 static int oracle_ce_row(const float *x, int64_t V, int64_t y,
-                         int64_t ignore_index, double st[4])
+                         int64_t ignore_index, double st[4], double *s_out)
 {
     st[0] = st[1] = st[2] = st[3] = 0.0;
+    if (s_out)
+        *s_out = 0.0;
     if (y == ignore_index)
         return ORACLE_ROW_IGNORED;
     if (y < 0 || y >= V)
@@ -130,14 +136,17 @@ static int oracle_ce_row(const float *x, int64_t V, int64_t y,
     for (int64_t j = 0; j < V; ++j)
         if ((double)x[j] > m)
             m = (double)x[j];
-    double d = 0.0;
+    double s = 0.0;
     for (int64_t j = 0; j < V; ++j)
-        d += exp((double)x[j] - m);
+        if (j != y)
+            s += exp((double)x[j] - m);
     double xy = (double)x[y];
     st[0] = m;
-    st[1] = d;
+    st[1] = s + exp(xy - m);
     st[2] = xy;
-    st[3] = m + log(d) - xy;
+    st[3] = log1p(s * exp(m - xy));
+    if (s_out)
+        *s_out = s;
     return ORACLE_ROW_VALID;
 }
 
@@ -152,7 +161,7 @@ void oracle_ce_fwd(const float *logits, const int64_t *target, int64_t M,
     for (int64_t r = 0; r < n_rows; ++r) {
         int64_t i = rows ? rows[r] : r;
         int c = oracle_ce_row(logits + i * V, V, target[i], ignore_index,
-                              stats + r * 4);
+                              stats + r * 4, NULL);
         if (row_code)
             row_code[r] = c;
     }
@@ -166,7 +175,9 @@ void oracle_ce_fwd(const float *logits, const int64_t *target, int64_t M,
 
 /* d loss_i / d x_ij = softmax(x_i)_j - [j == y_i], scaled by the upstream
  * gradient g_i = grad_loss[i * grad_stride] (stride 0: one scalar).
- * softmax_j = exp(x_j - m) / d with m, d recomputed here from the logits.
+ * softmax_j = exp(x_j - m) / d with m, d recomputed here from the logits; at
+ * the target, softmax_y - 1 = -s / d (s: the other columns' share, as in
+ * oracle_ce_row), the same value without the cancellation of 1 - 1.
  * Ignored and bad-target rows have gradient exactly 0. */
 void oracle_ce_bwd(const float *logits, const int64_t *target,
                    const float *grad_loss, int64_t grad_stride, int64_t M,
@@ -179,8 +190,8 @@ void oracle_ce_bwd(const float *logits, const int64_t *target,
         int64_t i = rows ? rows[r] : r;
         const float *x = logits + i * V;
         double *out = dlogits + r * V;
-        double st[4];
-        int c = oracle_ce_row(x, V, target[i], ignore_index, st);
+        double st[4], s;
+        int c = oracle_ce_row(x, V, target[i], ignore_index, st, &s);
         if (c != ORACLE_ROW_VALID) {
             for (int64_t j = 0; j < V; ++j)
                 out[j] = 0.0;
@@ -188,11 +199,8 @@ void oracle_ce_bwd(const float *logits, const int64_t *target,
         }
         double g = (double)grad_loss[i * grad_stride];
         int64_t y = target[i];
-        for (int64_t j = 0; j < V; ++j) {
-            double p = exp((double)x[j] - st[0]) / st[1];
-            double onehot = (j == y) ? 1.0 : 0.0;
-            out[j] = (p - onehot) * g;
-        }
+        for (int64_t j = 0; j < V; ++j)
+            out[j] = (j == y ? -s / st[1] : exp((double)x[j] - st[0]) / st[1]) * g;
     }
 }
 

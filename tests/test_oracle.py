@@ -253,6 +253,42 @@ def test_ce_bwd_two_value_closed_form_and_finite_difference():
         assert abs(fd - d[j]) < 1e-6
 
 
+def _decimal_row(x, y):
+    """-log softmax(x)_y and softmax(x)_y - 1 of one row in 60-digit decimal
+    arithmetic (exp and ln of the decimal module), as FP64."""
+    import decimal
+    ctx = decimal.Context(prec=60)
+    xs = [decimal.Decimal(float(v)) for v in x]   # exact: every FP32 value is a short decimal
+    m = max(xs)
+    e = [ctx.exp(ctx.subtract(v, m)) for v in xs]
+    d = decimal.Decimal(0)
+    for v in e:
+        d = ctx.add(d, v)
+    loss = ctx.ln(ctx.divide(d, e[y]))
+    grad_y = ctx.subtract(ctx.divide(e[y], d), decimal.Decimal(1))
+    return float(loss), float(grad_y)
+
+
+@pytest.mark.parametrize("gap", [0.0, 10.0, 25.0, 40.0, 70.0])
+def test_ce_confident_rows_against_decimal_arithmetic(gap):
+    """Rows whose target holds nearly all of the mass (the other columns
+    `gap` below it, losses from ~1e-2 down to ~1e-28): the loss and the
+    target's gradient keep full relative precision against 60-digit decimal
+    arithmetic, where m + log(d) - x_y and softmax_y - 1 would cancel."""
+    rng = np.random.default_rng(int(gap) + 3)
+    V, y = 300, 17
+    x = (rng.normal(0, 1, size=V) - gap).astype(np.float32)
+    x[y] = np.float32(2.5)
+    st, code = oracle.ce_fwd(x[None, :], np.array([y]))
+    d = oracle.ce_bwd(x[None, :], np.array([y]), 1.0)
+    loss, grad_y = _decimal_row(x, y)
+    assert code[0] == oracle.ROW_VALID
+    assert abs(st[0, 3] - loss) <= 1e-13 * abs(loss)
+    assert abs(d[0, y] - grad_y) <= 1e-13 * abs(grad_y)
+    # and the other entries still sum with it to zero
+    assert abs(d[0].sum()) <= 1e-12 * abs(grad_y) + 1e-300
+
+
 # --------------------------------------------------------------------------
 # a4/a5 gradient GEMMs
 # --------------------------------------------------------------------------
