@@ -92,7 +92,10 @@ LMH_API lmh_status_t lmhead_fwd(const void *X, const void *W, void *logits, int3
  *   logits  [M,V] FP32.   target [M] int64.
  *   stats   [M,4] FP32, per row {m, d, x_y, loss}:
  *             m = max_j x_j, d = sum_j exp(x_j - m), x_y = x[target],
- *             loss = m + log(d) - x_y  (= -log softmax(x)_target).
+ *             loss = -log softmax(x)_target = m + log(d) - x_y, computed as
+ *             log1p(s exp(m - x_y)) with s = d - exp(x_y - m) summed over the
+ *             other columns, so that it keeps its precision when the target
+ *             holds nearly all of the row's mass.
  *   A row whose target equals ignore_index is not read and gets
  *   {0,0,0,0}.  A target outside [0,V) that is not ignore_index sets
  *   LMH_DEV_BAD_TARGET in *status and the row is treated as ignored.
@@ -109,7 +112,9 @@ LMH_API lmh_status_t ce_fwd(const float *logits, const int64_t *target, float *s
  *              grad_loss_stride 0 = one scalar for every row,
  *              1 = one value per row ([M]); anything else is unsupported.
  *   dlogits    [M,V], dl_dtype LMH_F32 or LMH_BF16 (round to nearest even):
- *              dl[i,j] = (exp(x_ij - m_i) / d_i - [j == target_i]) * g_i.
+ *              dl[i,j] = (exp(x_ij - m_i) / d_i - [j == target_i]) * g_i;
+ *              at the target, softmax - 1 = exp(-loss_i) - 1 is taken as
+ *              expm1(-loss_i) from the saved loss (no cancellation).
  *              Ignored and bad-target rows are written as zeros.
  *              With LMH_F32, dlogits may be the logits buffer itself
  *              (in-place; each element is read before it is overwritten).
@@ -121,7 +126,8 @@ LMH_API lmh_status_t ce_bwd(const float *logits, const int64_t *target, const fl
 
 /* logits = X . W^T (FP32) and the cross-entropy forward statistics of those
  * logits in one pass over them: the vocabulary GEMM's epilogue reduces every
- * 128-wide vocabulary block of each token row to a partial (max, sum-exp) in
+ * 128-wide vocabulary block of each token row to a partial (max, sum-exp,
+ * the sum leaving out the target's own term) in
  * `workspace` and records the target logit while the tile is still on chip,
  * and a second kernel merges each token's partials (in a fixed order) into
  * stats[M,4] = {m, d, x_y, loss}.  The logits are written but not read back
@@ -180,7 +186,9 @@ LMH_API lmh_status_t lmhead_fwd_ce_noalloc(const void *X, const void *W, const i
  * all-gather of the [M,4] shard records) is the caller's.
  *
  * ce_fwd_shard: per row of this shard, shard_stats[M,4] = {m_r, d_r, x_y or 0,
- *   1 if the target is in this shard else 0}; ignored rows (target ==
+ *   1 if the target is in this shard else 0}: m_r = the max over the shard's
+ *   columns, d_r = sum of exp(x - m_r) over them, leaving out the target's own
+ *   term in the shard that holds it; ignored rows (target ==
  *   ignore_index) and bad targets (outside [0, vocab_total)) give zeros, bad
  *   targets also set LMH_DEV_BAD_TARGET.
  *   Requirements: 0 <= vocab_offset, vocab_offset + V <= vocab_total. */
@@ -190,17 +198,18 @@ LMH_API lmh_status_t ce_fwd_shard(const float *logits, const int64_t *target, fl
 
 /* ce_merge_shards: stats[M,4] = {m, d, x_y, loss} of the whole vocabulary
  * from the num_shards records of every shard, laid out shard-major
- * (shard_stats[r][M][4]): m = max_r m_r, d = sum_r d_r exp(m_r - m) taken in
- * shard order (deterministic), x_y from the owning shard,
- * loss = (m - x_y) + log d.  The result is what ce_fwd gives on the whole
- * rows, up to the order of the sums. */
+ * (shard_stats[r][M][4]): m = max_r m_r, s = sum_r d_r exp(m_r - m) taken in
+ * shard order (deterministic; every column but the target), x_y from the
+ * owning shard, d = s + exp(x_y - m), loss = log1p(s exp(m - x_y)).  The
+ * result is what ce_fwd gives on the whole rows, up to the order of the sums. */
 LMH_API lmh_status_t ce_merge_shards(const float *shard_stats, int64_t num_shards,
                                      const int64_t *target, float *stats, int64_t M,
                                      int64_t vocab_total, int64_t ignore_index, int32_t *status,
                                      lmh_stream_t stream);
 
 /* ce_bwd_shard: ce_bwd on a shard, with the merged stats: dl[i,j] =
- * (exp(x_ij - m_i) / d_i - [vocab_offset + j == target_i]) * g_i. */
+ * (exp(x_ij - m_i) / d_i - [vocab_offset + j == target_i]) * g_i, the target's
+ * entry as in ce_bwd. */
 LMH_API lmh_status_t ce_bwd_shard(const float *logits, const int64_t *target, const float *stats,
                                   const float *grad_loss, int64_t grad_loss_stride, void *dlogits,
                                   int32_t dl_dtype, int64_t M, int64_t V, int64_t vocab_offset,

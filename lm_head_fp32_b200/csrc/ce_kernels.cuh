@@ -10,6 +10,12 @@
 // stride over rows, so any grid works), 128-bit read-only streaming loads, an
 // online (max, sum-exp) pair per thread merged by warp shuffles and then
 // across warps in shared memory.
+//
+// The forward sums exp(x_j - m) over every column but the target (dx) and
+// adds the target's term only at the end: the loss log1p(dx * exp(m - x_y))
+// and, in the backward, the target's gradient (softmax_y - 1) g =
+// expm1(-loss) g then keep their precision on rows whose target holds nearly
+// all of the mass, where 1/d - 1 in FP32 would cancel to 0.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -112,14 +118,25 @@ __device__ __forceinline__ int row_kind(int64_t y, int64_t V, int64_t ignore_ind
     return 0;
 }
 
+// Component c of a loaded float4 replaced by -inf (the target's column, left
+// out of the running pair).
+__device__ __forceinline__ void mask_lane(float4 &a, int c)
+{
+    a.x = c == 0 ? -INFINITY : a.x;
+    a.y = c == 1 ? -INFINITY : a.y;
+    a.z = c == 2 ? -INFINITY : a.z;
+    a.w = c == 3 ? -INFINITY : a.w;
+}
+
 // stats[row] = {m, d, x_y, loss}.  VEC: V % 4 == 0 and logits 16-byte aligned.
 // The rows hold vocabulary entries [voff, voff + V) of a vocabulary of Vtot
 // (voff = 0, Vtot = V for a whole row); targets are global ids.  SHARD: the
 // rows are one shard of a vocabulary split across devices, and the record is
 // {m, d, x_y or 0, 1 if the target lies in this shard else 0} for
-// ce_merge_shards_kernel to combine.
+// ce_merge_shards_kernel to combine, where the shard that owns the target
+// leaves the target's term out of d (and still counts x_y in m).
 template <bool VEC, int THREADS = 512, bool SHARD = false>
-__global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict__ logits,
+__global__ void __launch_bounds__(THREADS, 2048 / THREADS) ce_fwd_kernel(const float *__restrict__ logits,
                                                             const int64_t *__restrict__ target,
                                                             float4 *__restrict__ stats, int64_t M,
                                                             int64_t V, int64_t ignore_index,
@@ -153,34 +170,50 @@ __global__ void __launch_bounds__(THREADS) ce_fwd_kernel(const float *__restrict
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
             const int64_t n4 = V >> 2;
             int64_t i = threadIdx.x;
+            // the one thread whose vectors include the target's leaves it out
+            const int64_t iy = owner ? (yl >> 2) : -1;
+            const bool has_y = owner && (iy % THREADS) == threadIdx.x;
+            const int cy = static_cast<int>(yl & 3);
             // four independent 128-bit loads in flight per thread per step
             for (; i + 3 * THREADS < n4; i += 4 * THREADS) {
                 float4 a = ldg_stream(x4 + i), b = ldg_stream(x4 + i + THREADS),
                        c = ldg_stream(x4 + i + 2 * THREADS),
                        e = ldg_stream(x4 + i + 3 * THREADS);
+                if (has_y) {
+                    if (i == iy) mask_lane(a, cy);
+                    if (i + THREADS == iy) mask_lane(b, cy);
+                    if (i + 2 * THREADS == iy) mask_lane(c, cy);
+                    if (i + 3 * THREADS == iy) mask_lane(e, cy);
+                }
                 const float v[16] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w,
                                      c.x, c.y, c.z, c.w, e.x, e.y, e.z, e.w};
                 fold<16>(s, v);
             }
             for (; i < n4; i += THREADS) {
                 float4 a = ldg_stream(x4 + i);
+                if (has_y && i == iy)
+                    mask_lane(a, cy);
                 const float v[4] = {a.x, a.y, a.z, a.w};
                 fold<4>(s, v);
             }
         } else {
             for (int64_t j = threadIdx.x; j < V; j += THREADS)
-                fold1(s, ldg_stream1(x + j));
+                if (j != yl)
+                    fold1(s, ldg_stream1(x + j));
         }
         s = block_merge(s, red);
         if (threadIdx.x == 0) {
-            if (SHARD) {
-                stats[row] = make_float4(s.m, s.d, xy, owner ? 1.f : 0.f);
-            } else {
-                // (m - x_y) first: exact when x_y is the maximum, so a near-zero
-                // loss is not swamped by the rounding of m + log(d).
-                const float loss = (s.m - xy) + logf(s.d);
-                stats[row] = make_float4(s.m, s.d, xy, loss);
+            // (m, dx) over every column but the target; the target joins the
+            // maximum here
+            float m = s.m, dx = s.d;
+            if (owner && xy > m) {
+                dx = m == -INFINITY ? 0.f : dx * exp_neg(m - xy);
+                m = xy;
             }
+            if (SHARD)
+                stats[row] = make_float4(m, dx, xy, owner ? 1.f : 0.f);
+            else
+                stats[row] = make_float4(m, ce_full_sum(m, dx, xy), xy, ce_loss(m, dx, xy));
         }
     }
 }
@@ -209,7 +242,11 @@ __device__ __forceinline__ void store1(float *p, float a) { *p = a; }
 __device__ __forceinline__ void store1(__nv_bfloat16 *p, float a) { *p = __float2bfloat16_rn(a); }
 
 // dl[row, j] = (exp(x - m) / d - [j == y]) * g, FP32 arithmetic, rounded to
-// OutT only at the store.  Ignored / bad-target rows are written as zeros.
+// OutT only at the store; at the target, softmax_y - 1 = exp(-loss) - 1 is
+// taken as expm1(-loss) from the saved loss, so that it does not cancel when
+// softmax_y is close to 1 (the thread that stored the target's entry with the
+// rest of its vector overwrites it).  Ignored / bad-target rows are written
+// as zeros.
 // VEC: V % 4 == 0, logits 16-byte and dl (4 * sizeof(OutT))-byte aligned.
 // Each element is read before it is written, by the same thread, so dl may
 // alias logits when OutT is float (ALIAS: coherent loads instead of the
@@ -217,7 +254,7 @@ __device__ __forceinline__ void store1(__nv_bfloat16 *p, float a) { *p = __float
 // The rows hold vocabulary entries [voff, voff + V) of a vocabulary of Vtot
 // (a shard when voff > 0 or V < Vtot): the one-hot is at the global target.
 template <typename OutT, bool VEC, bool ALIAS, int THREADS = 512>
-__global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
+__global__ void __launch_bounds__(THREADS, 2048 / THREADS) ce_bwd_kernel(
     const float *logits, const int64_t *__restrict__ target, const float4 *__restrict__ stats,
     const float *__restrict__ grad_loss, int64_t grad_stride, OutT *dl, int64_t M, int64_t V,
     int64_t ignore_index, int32_t *status, int64_t voff, int64_t Vtot)
@@ -249,7 +286,10 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
             continue;
         }
         const float m = st.x;
-        const float inv_d = 1.0f / st.y;
+        const float gd = g / st.y;  // g / d: softmax_j g = exp(x_j - m) gd
+        // the thread that stores the target's entry with the rest of its vector
+        const bool own_y = y >= 0 && y < V && ((VEC ? (y >> 2) : y) % THREADS) == threadIdx.x;
+        const float gy = own_y ? expm1f(-st.w) * g : 0.f;
         if (VEC) {
             const float4 *x4 = reinterpret_cast<const float4 *>(x);
             const int64_t n4 = V >> 2;
@@ -261,34 +301,30 @@ __global__ void __launch_bounds__(THREADS) ce_bwd_kernel(
                 for (int u = 0; u < 4; ++u)
                     a[u] = load4<ALIAS>(x4 + i + u * THREADS);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t ja = 4 * (i + u * THREADS);
-                    store4<OutT>(o + ja, (exp_neg(a[u].x - m) * inv_d - (ja + 0 == y)) * g,
-                                 (exp_neg(a[u].y - m) * inv_d - (ja + 1 == y)) * g,
-                                 (exp_neg(a[u].z - m) * inv_d - (ja + 2 == y)) * g,
-                                 (exp_neg(a[u].w - m) * inv_d - (ja + 3 == y)) * g);
-                }
+                for (int u = 0; u < 4; ++u)
+                    store4<OutT>(o + 4 * (i + u * THREADS), exp_neg(a[u].x - m) * gd,
+                                 exp_neg(a[u].y - m) * gd, exp_neg(a[u].z - m) * gd,
+                                 exp_neg(a[u].w - m) * gd);
             }
             for (; i < n4; i += THREADS) {
                 const float4 a = load4<ALIAS>(x4 + i);
-                const int64_t ja = 4 * i;
-                store4<OutT>(o + ja, (exp_neg(a.x - m) * inv_d - (ja + 0 == y)) * g,
-                             (exp_neg(a.y - m) * inv_d - (ja + 1 == y)) * g,
-                             (exp_neg(a.z - m) * inv_d - (ja + 2 == y)) * g,
-                             (exp_neg(a.w - m) * inv_d - (ja + 3 == y)) * g);
+                store4<OutT>(o + 4 * i, exp_neg(a.x - m) * gd, exp_neg(a.y - m) * gd,
+                             exp_neg(a.z - m) * gd, exp_neg(a.w - m) * gd);
             }
         } else {
-            for (int64_t j = threadIdx.x; j < V; j += THREADS) {
-                const float v = load1<ALIAS>(x + j);
-                store1(o + j, (exp_neg(v - m) * inv_d - (j == y)) * g);
-            }
+            for (int64_t j = threadIdx.x; j < V; j += THREADS)
+                store1(o + j, exp_neg(load1<ALIAS>(x + j) - m) * gd);
         }
+        // the target's entry, over the one stored above (program order)
+        if (own_y)
+            store1(o + y, gy);
     }
 }
 
 // stats[i] = {m, d, x_y, loss} from R shard records (ce_fwd_kernel with
 // SHARD) laid out shard-major, shard_stats[r * M + i]: the pairs are merged
-// in shard order and x_y comes from the shard that owns the target.
+// in shard order (their sums leave out the target's term, which the owning
+// shard dropped) and x_y comes from the shard that owns the target.
 __global__ void __launch_bounds__(256)
     ce_merge_shards_kernel(const float4 *__restrict__ shard_stats, int64_t R,
                            const int64_t *__restrict__ target, float4 *__restrict__ stats, int64_t M,
@@ -313,7 +349,7 @@ __global__ void __launch_bounds__(256)
             if (q.w != 0.f)
                 xy = q.z;
         }
-        stats[i] = make_float4(s.m, s.d, xy, (s.m - xy) + logf(s.d));
+        stats[i] = make_float4(s.m, ce_full_sum(s.m, s.d, xy), xy, ce_loss(s.m, s.d, xy));
     }
 }
 
@@ -383,8 +419,9 @@ __global__ void __launch_bounds__(WARPS * 32)
             if (kind == 2 && status)
                 atomicOr(status, 1);
         } else {
+            // the partials leave out the target's term (see ce_subtile_stats)
             const float xy = reinterpret_cast<const float *>(stats)[tok * 4 + 2];
-            stats[tok] = make_float4(r.m, r.d, xy, (r.m - xy) + logf(r.d));
+            stats[tok] = make_float4(r.m, ce_full_sum(r.m, r.d, xy), xy, ce_loss(r.m, r.d, xy));
         }
     }
 }

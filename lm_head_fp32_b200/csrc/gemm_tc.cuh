@@ -189,16 +189,21 @@ __host__ __device__ inline void tile_coords(int t, const GemmParams &p, int &mt,
 // Partial cross-entropy statistics of one staged sub-tile (FP32 logits):
 // lane l takes token row l of the 32 x 32 box in shared memory (32 vocabulary
 // columns starting at vbase; columns at or past V excluded) and returns its
-// (max, sum of exp(x - max)); the lane whose row holds its token's target
-// column also records the target logit.  Lanes without a token return the
-// empty pair.  The row is read as eight 16-byte chunks, lane l starting at
-// chunk l mod 8, so the eight lanes of each quarter-warp read eight different
-// bank groups; max and sum do not depend on the order the values are held in.
+// (max, sum of exp(x - max)), the sum over every column but the token's
+// target (which counts in the max; the finalize adds its term, so that the
+// loss keeps its precision when the target holds nearly all of the mass);
+// the lane whose row holds its token's target column also records the target
+// logit.  Lanes without a token return the empty pair.  The row is read as
+// eight 16-byte chunks, lane l starting at chunk l mod 8, so the eight lanes
+// of each quarter-warp read eight different bank groups; max and sum do not
+// depend on the order the values are held in.
 __device__ __forceinline__ MaxSum ce_subtile_stats(const float *buf, int lane, int rows, int vbase,
                                                    int V, int tok, int ntok, const GemmParams &p)
 {
     if (lane >= rows || tok >= ntok)
         return MaxSum{-INFINITY, 0.f};
+    const int64_t y = p.ce_target[tok];
+    const int yc = (y >= vbase && y < vbase + 32 && y < V) ? static_cast<int>(y - vbase) : -1;
     const float *rowp = buf + lane * 32;
     const float4 *row4 = reinterpret_cast<const float4 *>(rowp);
     const int nvalid = V - vbase;  // may be <= 0 (a slice past the vocabulary) or > 32
@@ -228,13 +233,24 @@ __device__ __forceinline__ MaxSum ce_subtile_stats(const float *buf, int lane, i
         vmax = fmaxf(vmax, v[i]);
     float dsum = 0.f;
     if (vmax != -INFINITY) {
+        if (yc < 0) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            dsum += exp_neg_ftz(v[i] - vmax);  // a masked column adds exp(-inf) = 0
+            for (int i = 0; i < 32; ++i)
+                dsum += exp_neg_ftz(v[i] - vmax);  // a masked column adds exp(-inf) = 0
+        } else {
+            // the block of this token's target (one in V / 32 of them)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int c = (kk + lane) & 7;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (4 * c + e != yc)
+                        dsum += exp_neg_ftz(v[4 * kk + e] - vmax);
+            }
+        }
     }
-    const int64_t y = p.ce_target[tok];
-    if (y >= vbase && y < vbase + 32 && y < V)
-        p.ce_stats[static_cast<int64_t>(tok) * 4 + 2] = rowp[y - vbase];
+    if (yc >= 0)
+        p.ce_stats[static_cast<int64_t>(tok) * 4 + 2] = rowp[yc];
     return MaxSum{vmax, dsum};
 }
 

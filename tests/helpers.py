@@ -145,7 +145,10 @@ class FakeOps:
                 continue
             m = x[i].max()
             own = off <= y < off + V
-            r[i] = (m, np.exp(x[i] - m).sum(), x[i, y - off] if own else 0.0, 1.0 if own else 0.0)
+            e = np.exp(x[i] - m)
+            # the shard that owns the target leaves its term out of the sum
+            dx = np.delete(e, y - off).sum() if own else e.sum()
+            r[i] = (m, dx, x[i, y - off] if own else 0.0, 1.0 if own else 0.0)
         rec.copy_(torch.from_numpy(r).float())
 
     @staticmethod
@@ -156,9 +159,9 @@ class FakeOps:
             if y == ignore or y < 0 or y >= vtot:
                 continue
             m = R[:, i, 0].max()
-            d = (R[:, i, 1] * np.exp(R[:, i, 0] - m)).sum()
+            dx = (R[:, i, 1] * np.exp(R[:, i, 0] - m)).sum()   # every column but the target
             xy = R[R[:, i, 3] != 0, i, 2].sum()
-            out[i] = (m, d, xy, m + np.log(d) - xy)
+            out[i] = (m, dx + np.exp(xy - m), xy, np.log1p(dx * np.exp(m - xy)))
         stats.copy_(torch.from_numpy(out).float())
 
     @staticmethod
@@ -171,7 +174,7 @@ class FakeOps:
                 continue
             out[i] = np.exp(x[i] - st[i, 0]) / st[i, 1]
             if off <= y < off + x.shape[1]:
-                out[i, y - off] -= 1.0
+                out[i, y - off] = np.expm1(-st[i, 3])   # softmax_y - 1 = exp(-loss) - 1
             out[i] *= float(g.reshape(-1)[0])
         dl.copy_(torch.from_numpy(out).to(dl.dtype))
 
