@@ -64,14 +64,18 @@ struct GemmParams {
     int32_t l2_out;     // L2 policy of the output stores (TMA store epilogue): 0 none, 1 evict first
     int32_t *status;
     uint64_t wait_limit_ns;  // limit of every pipeline wait (the host sets kWaitLimitNs)
-    // The last split_tiles tiles of the tile order are each computed as two
-    // work items, the first and the second half of the k-blocks (all first
-    // halves, then all second halves), whose FP32 sums are both added (TMA
-    // reduce-add, or atomic adds on the direct-store path) into output the
-    // host has zeroed: fl(0 + a) = a and fl(a + b) = fl(b + a), so the result
-    // does not depend on which half lands first.  0 = no split (requires two
-    // or more k-blocks).
+    // The last split_tiles tiles of the tile order (the last wave, which
+    // would leave units idle) are each computed as two work items: a long part,
+    // k-blocks [0, split_kb), on the unit that would have run the tile, and a
+    // short part, [split_kb, num_kb), on one of the units the wave leaves
+    // idle, each of which runs split_rounds short parts in turn.  Both parts'
+    // FP32 sums are added (TMA reduce-add, or atomic adds on the direct-store
+    // path) into output the host has zeroed: fl(0 + a) = a and fl(a + b) =
+    // fl(b + a), so the result does not depend on which part lands first.
+    // 0 = no split; the tiles before the split ones fill whole waves.
     int32_t split_tiles;
+    int32_t split_kb;
+    int32_t split_rounds;
     int32_t allow_split;  // host side: the call may split its last wave (FP32 output)
     // fused cross-entropy statistics (vocabulary GEMM only): per 128-wide
     // vocabulary block s (one CTA's rows of a tile) and token i,
@@ -306,24 +310,38 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
     const int num_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int num_tiles = p.num_m_tiles * p.num_n_tiles;
     const int num_kb = (p.Kdim + kBlockK - 1) / kBlockK;
-    const int split_first = num_tiles - p.split_tiles;
-    const int num_items = split_first + 2 * p.split_tiles;
-    // work item -> tile and k-block range [kb0, kb1); true for a half tile
-    auto item_of = [&](int it, int &t, int &kb0, int &kb1) -> bool {
+    const int split_first = num_tiles - p.split_tiles;  // a whole number of waves
+    const int num_items = split_first + (p.split_tiles > 0 ? num_units * p.split_rounds : 0);
+    // work item -> tile and k-block range [kb0, kb1): 0 a whole tile, 1 a part
+    // of a split tile, -1 no work (every role skips the same items).  Past
+    // split_first, item it belongs to unit (it - split_first) % num_units.
+    auto item_of = [&](int it, int &t, int &kb0, int &kb1) -> int {
         if (it < split_first) {
             t = it;
             kb0 = 0;
             kb1 = num_kb;
-            return false;
+            return 0;
         }
-        // every split tile's first half, then every second half (all of them
-        // run in the same wave)
         const int j = it - split_first;
-        const bool second = j >= p.split_tiles;
-        t = split_first + (second ? j - p.split_tiles : j);
-        kb0 = second ? num_kb / 2 : 0;
-        kb1 = second ? num_kb : num_kb / 2;
-        return true;
+        const int r = j / num_units;       // round of the last wave
+        const int u = j - r * num_units;   // the unit
+        if (u < p.split_tiles) {
+            // the long part of the tile this unit would have run
+            if (r != 0)
+                return -1;
+            t = split_first + u;
+            kb0 = 0;
+            kb1 = p.split_kb;
+            return 1;
+        }
+        // the units the wave leaves idle take the short parts, round by round
+        const int idx = (u - p.split_tiles) + r * (num_units - p.split_tiles);
+        if (idx >= p.split_tiles)
+            return -1;
+        t = split_first + idx;
+        kb0 = p.split_kb;
+        kb1 = num_kb;
+        return 1;
     };
 
     if (threadIdx.x == 0) {
@@ -417,7 +435,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
             bool ok = true;
             for (int it = unit; it < num_items && ok; it += num_units) {
                 int t, kb0, kb1, mt, nt;
-                item_of(it, t, kb0, kb1);
+                if (item_of(it, t, kb0, kb1) < 0)
+                    continue;
                 tile_coords(t, p, mt, nt);
                 const int m0 = mt * C::TILE_M + static_cast<int>(rank) * kBlockM;  // this CTA's A rows
                 const int nb0 = nt * BN + static_cast<int>(rank) * C::BN_CTA;     // this CTA's B rows
@@ -444,7 +463,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
             bool ok = true;
             for (int it = unit; it < num_items && ok; it += num_units) {
                 int t, kb0, kb1;
-                item_of(it, t, kb0, kb1);
+                if (item_of(it, t, kb0, kb1) < 0)
+                    continue;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns)) {
                     ok = false;
                     break;
@@ -518,14 +538,17 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
         const uint32_t empty_addr0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
         uint32_t acc = 0, acc_phase = 0;
         for (int it = unit; it < num_items; it += num_units) {
+            int t, kb0, kb1, mt, nt;
+            const int kind = item_of(it, t, kb0, kb1);
+            if (kind < 0)
+                continue;
+            const bool part = kind == 1;  // one of two addends of a split tile
             // every lane waits, then the warp agrees, so the .sync.aligned
             // tensor-memory loads below always run with the full warp
             const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok))
                 break;
             tc_fence_after();
-            int t, kb0, kb1, mt, nt;
-            const bool half_tile = item_of(it, t, kb0, kb1);
             tile_coords(t, p, mt, nt);
             const int mbase = mt * C::TILE_M + static_cast<int>(rank) * kBlockM;
             const int m = mbase + row;
@@ -552,7 +575,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        if (ACC || half_tile)
+                        if (ACC || part)
                             tma_reduce_add_2d(&tmC, buf, mbase + q * 32, n0 + c);
                         else if (p.l2_out)
                             tma_store_2d_hint(&tmC, buf, mbase + q * 32, n0 + c, pol_out);
@@ -607,7 +630,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, RES)
                     for (int j = 0; j < C::EPI_CHUNK; ++j)
                         if (n0 + c + j < p.Ndim) {
                             // FP32 only: an accumulating or half-tile store adds
-                            if (sizeof(OutT) == 4 && (ACC || half_tile))
+                            if (sizeof(OutT) == 4 && (ACC || part))
                                 atomicAdd(reinterpret_cast<float *>(o) + static_cast<int64_t>(j) * p.ldo,
                                           __uint_as_float(r[j]));
                             else

@@ -138,21 +138,35 @@ def test_sweep_corner_k16384_sampled(M):
     assert_bf16_close(out16[tr], ref, "BF16 logits", abs_tol=logits_tol(X, W))
 
 
-def _dx_split_tiles(M, K, V):
-    """Tiles of lmhead_bwd_dx split into two k-halves, as the library decides
-    for 256 x 256 CTA-pair tiles on (SMs / 2) pairs: those of a last (or only)
-    wave that fills at most half of the pairs."""
+def _dx_split(M, K, V):
+    """How lmhead_bwd_dx splits the last (or only) wave of 256 x 256 CTA-pair
+    tiles on (SMs / 2) pairs, restated: each of its rem tiles becomes a long
+    part [0, B) and a short part [B, num_kb), the pairs the wave leaves idle
+    taking k short parts each, B = ceil(num_kb k / (k + 1)); taken when the
+    last round shortens by a tenth, and for k > 1 only after a full wave.
+    Returns (rem, k, B) or None."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles, pairs = (-(-K // 256)) * (-(-M // 256)), sms // 2
-    rem = tiles % pairs
-    return rem if 0 < 2 * rem <= pairs else 0
+    nk, rem = -(-V // 64), tiles % pairs
+    if nk < 2 or rem == 0:
+        return None
+    k = -(-rem // (pairs - rem))
+    B = -(-nk * k // (k + 1))
+    if (k == 1 or tiles > pairs) and k <= 8 and B < nk and 10 * max(B, k * (nk - B)) <= 9 * nk:
+        return rem, k, B
+    return None
+
+
+def _dx_split_tiles(M, K, V):
+    s = _dx_split(M, K, V)
+    return s[0] if s else 0
 
 
 def test_dx_last_wave_split_integer_exact():
     """2560 tokens x K = 2048: 80 pair tiles, so on 74 SM pairs the last 6 are
-    computed as two k-halves added into zeroed output.  Integer operands keep
-    every partial sum exact, so the words must equal the oracle's; V = 1032
-    gives 17 k-blocks (halves of 8 and 9, the last one ragged)."""
+    each computed as two parts added into zeroed output.  Integer operands
+    keep every partial sum exact, so the words must equal the oracle's;
+    V = 1032 gives 17 k-blocks (parts of 9 and 8, the last one ragged)."""
     M, K, V = 2560, 2048, 1032
     if _dx_split_tiles(M, K, V) == 0:
         pytest.skip("this GPU's SM count does not split the last wave of this shape")
@@ -186,9 +200,9 @@ def test_dx_last_wave_split_random_deterministic():
 
 def test_dx_single_sparse_wave_split_integer_exact_and_deterministic():
     """Few tiles (a ragged token tile, 384 = 256 + 128, and K = 256: two pair
-    tiles) on many SM pairs: both tiles are split into k-halves, so four pairs
-    work.  V = 65544 gives 1025 k-blocks (halves of 512 and 513, the last one
-    ragged).  Integer operands keep the words exact; random operands are within
+    tiles) on many SM pairs: both tiles are split into two parts, so four
+    pairs work.  V = 65544 gives 1025 k-blocks (parts of 513 and 512, the last
+    one ragged).  Integer operands keep the words exact; random operands are within
     the tolerance and bitwise repeatable."""
     M, K, V = 384, 256, 65544
     assert _dx_split_tiles(M, K, V) == 2
@@ -202,6 +216,34 @@ def test_dx_single_sparse_wave_split_integer_exact_and_deterministic():
     rows = np.array([0, 1, 200, 255, 256, 300, M - 1])
     assert_abs_close(to_f64(out[torch.as_tensor(rows, device=DEV)]),
                      oracle.dx(bits(dl), bits(W), rows=rows), gemm_tol(V, dl, W), "dX split")
+    for _ in range(2):
+        assert torch.equal(out, gpu_dx(dl, W))
+
+
+@pytest.mark.parametrize("M,K,V,k", [(2048, 4096, 8200, 3), (4352, 1792, 4104, 2)])
+def test_dx_split_with_several_short_parts(M, K, V, k):
+    """A last wave that fills most of the SM pairs after a full one: 128
+    tiles (2048 tokens, K = 4096) leave 20 of 74 pairs idle in the second
+    round, so each of its 54 tiles keeps a long part of 97 of its 129 k-blocks
+    and the idle pairs take 3 short parts of 32 each; 119 tiles (4352 tokens,
+    K = 1792) take 2 short parts per idle pair.  Integer operands: the words
+    must equal the oracle's on sampled token rows (every output column, so
+    every tile of those rows); random operands: within the tolerance and
+    bitwise repeatable."""
+    plan = _dx_split(M, K, V)
+    if plan is None or plan[1] != k:
+        pytest.skip("this GPU's SM count gives another split of this shape")
+    rows = np.unique(np.concatenate([np.arange(0, M, 61), [M - 1]]))
+    tr = torch.as_tensor(rows, device=DEV)
+    dl = synth.int_bf16((M, V), 71)
+    W = synth.int_bf16((V, K), 72)
+    got = gpu_dx(dl, W)[tr].cpu().numpy()
+    assert np.array_equal(got, oracle.round_f32(oracle.dx(bits(dl), bits(W), rows=rows)))
+    dl = synth.normal_bf16((M, V), 1e-3, 73)
+    W = synth.normal_bf16((V, K), 0.02, 74)
+    out = gpu_dx(dl, W)
+    assert_abs_close(to_f64(out[tr]), oracle.dx(bits(dl), bits(W), rows=rows),
+                     gemm_tol(V, dl, W), "dX split")
     for _ in range(2):
         assert torch.equal(out, gpu_dx(dl, W))
 

@@ -2,7 +2,7 @@
 forward, against the FP64 oracle.  The shapes are drawn so that together they
 reach every GEMM variant the library picks by size: token tiles of 16, 32,
 64, 128 and 256 (single CTA, two CTAs per SM, and CTA pairs), ragged m, n and
-k tails, dX tiles split into two k-halves (a sparse wave) and unsplit, FP32
+k tails, dX tiles split into two parts (a sparse last wave) and unsplit, FP32
 and BF16 outputs.  Half of the cases use integer operands, for which every
 GEMM output must equal the oracle word for word."""
 import numpy as np
