@@ -10,6 +10,9 @@
 * The whole five-call step is captured in a CUDA graph and replayed: the calls
   only enqueue stream work (no allocation, no synchronisation), and replays
   reproduce the eager results bit for bit.
+* Two independent steps run at the same time on two streams (the library
+  holds no state between calls apart from cached driver handles) and give
+  the bits each gives alone; the dX split of the last wave is among them.
 """
 import pytest
 import torch
@@ -99,3 +102,48 @@ def test_whole_step_in_a_cuda_graph():
         for k in bufs:
             assert torch.equal(bufs[k], eager[k]), k
     del graph
+
+
+def _step_buffers(M, K, V, seed):
+    cfg = synth.GemmConfig(f"concurrent_{seed}", M, K, V, "normal", ignore_frac=0.02, seed=seed)
+    X, W, t = cfg.make()
+    g = torch.tensor([cfg.grad_scalar(t)], dtype=torch.float32, device=DEV)
+    ins = dict(X=X.to(DEV), W=W.to(DEV), t=t.to(DEV), g=g)
+    outs = dict(logits=guarded_empty((M, V)), stats=guarded_empty((M, 4)),
+                dl=guarded_empty((M, V), torch.bfloat16),
+                dX=guarded_empty((M, K)), dW=guarded_empty((V, K)))
+    return ins, outs
+
+
+def _run_step(ins, outs, status, stream):
+    lmhead.lmhead_fwd(ins["X"], ins["W"], outs["logits"], status, stream)
+    lmhead.ce_fwd(outs["logits"], ins["t"], outs["stats"], -100, status, stream)
+    lmhead.ce_bwd(outs["logits"], ins["t"], outs["stats"], ins["g"], outs["dl"], -100, status, stream)
+    lmhead.lmhead_bwd_dx(outs["dl"], ins["W"], outs["dX"], status, stream)
+    lmhead.lmhead_bwd_dw(outs["dl"], ins["X"], outs["dW"], status, stream)
+
+
+def test_two_streams_at_once_match_each_alone():
+    # 2560 tokens x K = 2048: dX's last wave is split (80 pair tiles on 74 pairs)
+    cases = [(2560, 2048, 1032, 5), (300, 1024, 8200, 6)]
+    bufs = [_step_buffers(*c) for c in cases]
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    alone = []
+    for ins, outs in bufs:
+        _run_step(ins, outs, status, None)
+        torch.cuda.synchronize()
+        alone.append({k: v.clone() for k, v in outs.items()})
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for _ in range(3):
+        for _, outs in bufs:
+            for v in outs.values():
+                v.zero_()
+        torch.cuda.synchronize()
+        for (ins, outs), s in zip(bufs, streams):
+            _run_step(ins, outs, status, s)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        for (_, outs), ref in zip(bufs, alone):
+            for k in outs:
+                assert torch.equal(outs[k], ref[k]), k
+
